@@ -1,0 +1,376 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each check compares the oracle with a closed form, a hand-worked fixture, a
+library routine, a 50-digit brute-force evaluation or an invariant, chosen so
+that a plausible slip in the oracle (a dropped term, a flipped sign or tap, a
+transposed B/C, an off-by-one in the recurrence, the skip term outside the gate)
+fails at least one of them.
+"""
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from mamba_selective_scan_sm_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _arr(x):
+    return None if x is None else np.asarray(x, dtype=np.float64)
+
+
+def _silu(v):
+    return v * scipy.special.expit(v)
+
+
+def _softplus(v):
+    return np.logaddexp(0.0, v)
+
+
+def _rand_case(rng, B=2, D=3, L=7, N=4, conv=0):
+    c = dict(u=rng.standard_normal((B, D, L)), delta=0.5 * rng.standard_normal((B, D, L)),
+             z=rng.standard_normal((B, D, L)), B=rng.standard_normal((B, N, L)),
+             C=rng.standard_normal((B, N, L)), A=-rng.uniform(0.2, 3.0, (D, N)),
+             D=rng.standard_normal(D), delta_bias=rng.uniform(-3, 0.5, D))
+    if conv:
+        c["conv_w"] = 0.5 * rng.standard_normal((D, conv))
+        c["conv_b"] = 0.3 * rng.standard_normal(D)
+    return c
+
+
+# ---------------------------------------------------------------- fixtures ---
+
+@pytest.mark.parametrize("name", ["l1_readout.json", "running_sum.json", "geometric_decay.json"])
+def test_golden_scan(name):
+    g = _golden(name)
+    tol = g.get("tolerance", 1e-15)
+    y, h = oracle.selective_scan(_arr(g["u"]), _arr(g["delta"]), _arr(g["A"]), _arr(g["B"]),
+                                 _arr(g["C"]), _arr(g["D"]), _arr(g["z"]), _arr(g["delta_bias"]),
+                                 g["delta_softplus"], False, return_final_state=True)
+    np.testing.assert_allclose(y, _arr(g["y"]), rtol=tol, atol=tol)
+    np.testing.assert_allclose(h, _arr(g["final_state"]), rtol=tol, atol=tol)
+    if "y_reverse" in g:
+        y, h = oracle.selective_scan(_arr(g["u"]), _arr(g["delta"]), _arr(g["A"]), _arr(g["B"]),
+                                     _arr(g["C"]), _arr(g["D"]), _arr(g["z"]),
+                                     _arr(g["delta_bias"]), g["delta_softplus"], True,
+                                     return_final_state=True)
+        np.testing.assert_allclose(y, _arr(g["y_reverse"]), rtol=tol, atol=tol)
+        np.testing.assert_allclose(h, _arr(g["final_state_reverse"]), rtol=tol, atol=tol)
+
+
+def test_golden_conv():
+    g = _golden("conv_orientation.json")
+    out = oracle.causal_conv1d(_arr(g["x"]), _arr(g["w"]), _arr(g["bias"]), g["apply_silu"])
+    np.testing.assert_array_equal(out, _arr(g["out"]))
+
+
+def test_golden_decode():
+    g = _golden("decode_step.json")
+    y, st, _ = oracle.state_update(_arr(g["state"]), None, _arr(g["x"]), _arr(g["dt"]),
+                                   _arr(g["A"]), _arr(g["B"]), _arr(g["C"]), _arr(g["D"]),
+                                   _arr(g["z"]), _arr(g["dt_bias"]), g["dt_softplus"])
+    np.testing.assert_array_equal(y, _arr(g["y"]))
+    np.testing.assert_array_equal(st, _arr(g["state_after"]))
+    # conv-state shift: newest input appended on the right
+    w = np.array([[0.25, 0.75]])
+    _, _, cs = oracle.state_update(_arr(g["state"]), _arr(g["conv_state"]), _arr(g["conv_x"]),
+                                   _arr(g["dt"]), _arr(g["A"]), _arr(g["B"]), _arr(g["C"]),
+                                   conv_w=w, conv_b=np.zeros(1), dt_softplus=False)
+    np.testing.assert_array_equal(cs, _arr(g["conv_state_after"]))
+
+
+# ------------------------------------------------------------ closed forms ---
+
+@pytest.mark.parametrize("softplus", [False, True])
+@pytest.mark.parametrize("gate", [False, True])
+def test_A_zero_is_running_sum(softplus, gate):
+    """A = 0: h_t = sum_{s<=t} delta_s B_s u_s (numpy cumsum), then y = C.h + D u, times silu(z)."""
+    rng = np.random.default_rng(1)
+    c = _rand_case(rng, B=2, D=3, L=37, N=5)
+    A0 = np.zeros_like(c["A"])
+    z = c["z"] if gate else None
+    y, h = oracle.selective_scan(c["u"], c["delta"], A0, c["B"], c["C"], c["D"], z,
+                                 c["delta_bias"], softplus, False, return_final_state=True)
+    dl = c["delta"] + c["delta_bias"][None, :, None]
+    if softplus:
+        dl = _softplus(dl)
+    dbu = dl[:, :, None, :] * c["B"][:, None, :, :] * c["u"][:, :, None, :]   # (B, D, N, L)
+    hs = np.cumsum(dbu, axis=-1)
+    yr = np.einsum("bnl,bdnl->bdl", c["C"], hs) + c["D"][None, :, None] * c["u"]
+    if gate:
+        yr = yr * _silu(c["z"])
+    np.testing.assert_allclose(y, yr, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h, hs[..., -1], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_constant_inputs_geometric_series(reverse):
+    """Constant delta, B, C, u: h_t = delta B u (1 - a^(k+1)) / (1 - a), a = exp(delta A),
+    k = number of steps taken before t."""
+    L, N = 50, 3
+    dl, Bv, Cv, uv, Dv = 0.37, np.array([0.7, -1.2, 2.0]), np.array([1.5, 0.4, -0.9]), 1.3, 0.6
+    A = np.array([[-0.5, -1.7, -3.1]])
+    u = np.full((1, 1, L), uv)
+    delta = np.full((1, 1, L), dl)
+    Bm = np.repeat(Bv[None, :, None], L, axis=2)
+    Cm = np.repeat(Cv[None, :, None], L, axis=2)
+    y, h = oracle.selective_scan(u, delta, A, Bm, Cm, np.array([Dv]), None, None, False, reverse,
+                                 return_final_state=True)
+    a = np.exp(dl * A[0])
+    k = np.arange(L)[::-1] if reverse else np.arange(L)
+    hs = dl * Bv[:, None] * uv * (1 - a[:, None] ** (k[None, :] + 1)) / (1 - a[:, None])
+    yr = (Cv[:, None] * hs).sum(0) + Dv * uv
+    np.testing.assert_allclose(y[0, 0], yr, rtol=1e-13)
+    np.testing.assert_allclose(h[0, 0], dl * Bv * uv * (1 - a ** L) / (1 - a), rtol=1e-13)
+
+
+def test_seqlen_one_readout():
+    """L = 1: y = (sum_n C_n delta B_n u + D u) silu(z), delta = softplus(dt + bias)."""
+    rng = np.random.default_rng(2)
+    c = _rand_case(rng, B=3, D=4, L=1, N=6)
+    y, h = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                 c["delta_bias"], True, False, return_final_state=True)
+    dl = _softplus(c["delta"][..., 0] + c["delta_bias"][None])
+    hr = dl[:, :, None] * c["B"][:, None, :, 0] * c["u"][..., 0][:, :, None]
+    yr = (np.einsum("bn,bdn->bd", c["C"][..., 0], hr) + c["D"][None] * c["u"][..., 0]) \
+        * _silu(c["z"][..., 0])
+    np.testing.assert_allclose(y[..., 0], yr, rtol=1e-13)
+    np.testing.assert_allclose(h, hr, rtol=1e-13)
+
+
+def test_softplus_zero_is_ln2_and_silu_zero_is_zero():
+    """delta = softplus(0) = ln 2 (A = 0, B = C = u = 1, N = 1: y = delta); silu(0) = 0 kills y."""
+    one = np.ones((1, 1, 1))
+    y = oracle.selective_scan(one, np.zeros((1, 1, 1)), np.zeros((1, 1)), one, one, None, None,
+                              np.zeros(1), True)
+    assert abs(y[0, 0, 0] - math.log(2.0)) < 1e-15
+    y = oracle.selective_scan(one, np.zeros((1, 1, 1)), np.zeros((1, 1)), one, one, None,
+                              np.zeros((1, 1, 1)), np.zeros(1), True)
+    assert y[0, 0, 0] == 0.0
+
+
+# -------------------------------------------------------- brute force, L<=8 ---
+
+def _mp_silu(v):
+    return v / (1 + mpmath.exp(-v))
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_bruteforce_50_digits(conv, reverse):
+    """h_t = sum_{s<=t} (prod_{r=s+1..t} dA_r) dBu_s as explicit products at 50 digits."""
+    mpmath.mp.dps = 50
+    rng = np.random.default_rng(3 + conv + int(reverse))
+    Bsz, D, L, N = 1, 2, 8, 3
+    c = _rand_case(rng, Bsz, D, L, N, conv=conv)
+    y = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                              c["delta_bias"], True, reverse, c.get("conv_w"), c.get("conv_b"))
+    for d in range(D):
+        x = [mpmath.mpf(float(v)) for v in c["u"][0, d]]
+        order = list(range(L))[::-1] if reverse else list(range(L))
+        xs = [x[t] for t in order]                     # sequence as the scan walks it
+        if conv:
+            w = [mpmath.mpf(float(v)) for v in c["conv_w"][d]]
+            us = []
+            for i in range(L):
+                acc = mpmath.mpf(float(c["conv_b"][d]))
+                for k in range(conv):
+                    s = i - (conv - 1) + k
+                    if s >= 0:
+                        acc += w[k] * xs[s]
+                us.append(_mp_silu(acc))
+        else:
+            us = xs
+        dts = [mpmath.log(1 + mpmath.exp(mpmath.mpf(float(c["delta"][0, d, t]))
+                                         + mpmath.mpf(float(c["delta_bias"][d])))) for t in order]
+        for i, t in enumerate(order):
+            yt = mpmath.mpf(0)
+            for n in range(N):
+                An = mpmath.mpf(float(c["A"][d, n]))
+                hn = mpmath.mpf(0)
+                for s in range(i + 1):
+                    prod = mpmath.mpf(1)
+                    for r in range(s + 1, i + 1):
+                        prod *= mpmath.exp(dts[r] * An)
+                    hn += prod * dts[s] * mpmath.mpf(float(c["B"][0, n, order[s]])) * us[s]
+                yt += mpmath.mpf(float(c["C"][0, n, t])) * hn
+            yt += mpmath.mpf(float(c["D"][d])) * us[i]
+            yt *= _mp_silu(mpmath.mpf(float(c["z"][0, d, t])))
+            assert abs(float(yt) - y[0, d, t]) <= 1e-13 * max(1.0, abs(float(yt))), (d, t)
+
+
+# ------------------------------------------------------ library routines ---
+
+@pytest.mark.parametrize("W", [2, 3, 4])
+def test_conv_matches_torch_conv1d(W):
+    """Depthwise Conv1d with padding W-1, first L outputs kept (the causal reading)."""
+    rng = np.random.default_rng(4)
+    Bsz, D, L = 2, 5, 19
+    x, w, b = rng.standard_normal((Bsz, D, L)), rng.standard_normal((D, W)), rng.standard_normal(D)
+    ref = torch.nn.functional.conv1d(torch.from_numpy(x), torch.from_numpy(w)[:, None, :],
+                                     torch.from_numpy(b), padding=W - 1, groups=D)[..., :L].numpy()
+    np.testing.assert_allclose(oracle.causal_conv1d(x, w, b, False), ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.causal_conv1d(x, w, b, True), _silu(ref), rtol=1e-12,
+                               atol=1e-12)
+
+
+def test_fused_conv_scan_equals_conv_then_scan():
+    rng = np.random.default_rng(5)
+    c = _rand_case(rng, 2, 3, 23, 4, conv=4)
+    y1 = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                               c["delta_bias"], True, False, c["conv_w"], c["conv_b"])
+    u = oracle.causal_conv1d(c["u"], c["conv_w"], c["conv_b"], True)
+    y2 = oracle.selective_scan(u, c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                               c["delta_bias"], True, False)
+    np.testing.assert_allclose(y1, y2, rtol=1e-14, atol=1e-14)
+
+
+# ------------------------------------------------------------- invariants ---
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_reverse_is_flip_forward_flip(conv):
+    rng = np.random.default_rng(6)
+    c = _rand_case(rng, 2, 3, 29, 4, conv=conv)
+    yr, hr = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                   c["delta_bias"], True, True, c.get("conv_w"), c.get("conv_b"),
+                                   return_final_state=True)
+    f = lambda a: None if a is None else a[..., ::-1]
+    yf, hf = oracle.selective_scan(f(c["u"]), f(c["delta"]), c["A"], f(c["B"]), f(c["C"]), c["D"],
+                                   f(c["z"]), c["delta_bias"], True, False, c.get("conv_w"),
+                                   c.get("conv_b"), return_final_state=True)
+    np.testing.assert_allclose(yr, yf[..., ::-1], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(hr, hf, rtol=1e-14, atol=1e-14)
+
+
+def test_decode_repeated_equals_scan():
+    """L decode steps from zero state and zero conv history reproduce the fused-conv scan."""
+    rng = np.random.default_rng(7)
+    Bsz, D, L, N, W = 2, 3, 17, 4, 4
+    c = _rand_case(rng, Bsz, D, L, N, conv=W)
+    y, h = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                 c["delta_bias"], True, False, c["conv_w"], c["conv_b"],
+                                 return_final_state=True)
+    st = np.zeros((Bsz, D, N))
+    cs = np.zeros((Bsz, D, W))
+    for t in range(L):
+        yt, st, cs = oracle.state_update(st, cs, c["u"][..., t], c["delta"][..., t], c["A"],
+                                         c["B"][..., t], c["C"][..., t], c["D"], c["z"][..., t],
+                                         c["delta_bias"], True, c["conv_w"], c["conv_b"])
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st, h, rtol=1e-12, atol=1e-13)
+
+
+def test_linear_in_u_without_conv_and_gate():
+    rng = np.random.default_rng(8)
+    c = _rand_case(rng, 1, 3, 31, 4)
+    u2 = rng.standard_normal(c["u"].shape)
+    run = lambda u: oracle.selective_scan(u, c["delta"], c["A"], c["B"], c["C"], c["D"], None,
+                                          c["delta_bias"], True)
+    np.testing.assert_allclose(run(2.5 * c["u"] - 0.75 * u2), 2.5 * run(c["u"]) - 0.75 * run(u2),
+                               rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_causality(reverse):
+    rng = np.random.default_rng(9)
+    c = _rand_case(rng, 1, 2, 40, 4, conv=4)
+    t0 = 17
+    run = lambda cc: oracle.selective_scan(cc["u"], cc["delta"], cc["A"], cc["B"], cc["C"], cc["D"],
+                                           cc["z"], cc["delta_bias"], True, reverse,
+                                           cc["conv_w"], cc["conv_b"])
+    y0 = run(c)
+    for key in ("u", "delta", "B", "C", "z"):
+        c2 = dict(c)
+        c2[key] = c[key].copy()
+        c2[key][..., t0] += 1.0
+        y1 = run(c2)
+        same = slice(t0 + 1, None) if reverse else slice(0, t0)
+        np.testing.assert_array_equal(y1[..., same], y0[..., same])
+        assert np.all(y1[..., t0] != y0[..., t0]) or key == "z", key
+
+
+def test_zero_B_or_C_leaves_skip_times_gate():
+    rng = np.random.default_rng(10)
+    c = _rand_case(rng, 2, 3, 13, 4)
+    ref = c["D"][None, :, None] * c["u"] * _silu(c["z"])
+    for kill in ("B", "C"):
+        cc = dict(c)
+        cc[kill] = np.zeros_like(c[kill])
+        y = oracle.selective_scan(cc["u"], cc["delta"], cc["A"], cc["B"], cc["C"], cc["D"], cc["z"],
+                                  cc["delta_bias"], True)
+        np.testing.assert_allclose(y, ref, rtol=1e-14, atol=1e-15)
+
+
+def test_conv_one_hot_taps():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((1, 2, 12))
+    w = np.zeros((2, 4))
+    w[:, 3] = 1.0                                   # newest tap: identity
+    np.testing.assert_array_equal(oracle.causal_conv1d(x, w, None, False), x)
+    w = np.zeros((2, 4))
+    w[:, 0] = 1.0                                   # oldest tap: shift by W-1, zero fill
+    out = oracle.causal_conv1d(x, w, None, False)
+    np.testing.assert_array_equal(out[..., 3:], x[..., :-3])
+    np.testing.assert_array_equal(out[..., :3], 0.0)
+
+
+def test_bidirectional_palindrome():
+    """Same parameters both ways and a palindromic sequence give a palindromic output."""
+    rng = np.random.default_rng(12)
+    c = _rand_case(rng, 1, 3, 21, 4, conv=4)
+    pal = lambda a: np.concatenate([a[..., :11], a[..., :10][..., ::-1]], axis=-1)
+    for k in ("u", "delta", "B", "C", "z"):
+        c[k] = pal(c[k])
+    y = oracle.selective_scan_bidir(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                    c["delta_bias"], c["A"], c["D"], c["delta_bias"], True,
+                                    c["conv_w"], c["conv_b"])
+    np.testing.assert_allclose(y, y[..., ::-1], rtol=1e-13, atol=1e-13)
+
+
+def test_two_pass_chunk_carry_matches_sequential():
+    """Chunk summaries (P_c = exp(A sum delta), S_c = state from zero), the carry
+    H_c = P_c H_{c-1} + S_c, and a rescan of each chunk from H_{c-1} give the
+    sequential result: the algebra the chunk-parallel GPU path relies on."""
+    rng = np.random.default_rng(13)
+    c = _rand_case(rng, 2, 3, 60, 4)
+    y, h = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                 c["delta_bias"], True, False, return_final_state=True)
+    bounds = [0, 13, 31, 32, 60]
+    H = np.zeros((2, 3, 4))
+    ys = []
+    for c0, c1 in zip(bounds[:-1], bounds[1:]):
+        sl = lambda a: a[..., c0:c1]
+        yc = oracle.selective_scan(sl(c["u"]), sl(c["delta"]), c["A"], sl(c["B"]), sl(c["C"]),
+                                   c["D"], sl(c["z"]), c["delta_bias"], True, False, h0=H)
+        _, S = oracle.selective_scan(sl(c["u"]), sl(c["delta"]), c["A"], sl(c["B"]), sl(c["C"]),
+                                     c["D"], sl(c["z"]), c["delta_bias"], True, False,
+                                     return_final_state=True)
+        dsum = _softplus(sl(c["delta"]) + c["delta_bias"][None, :, None]).sum(-1)
+        P = np.exp(dsum[..., None] * c["A"][None])
+        H = P * H + S
+        ys.append(yc)
+    np.testing.assert_allclose(np.concatenate(ys, axis=-1), y, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(H, h, rtol=1e-11, atol=1e-12)
+
+
+def test_oracle_consumes_bf16_rounded_inputs():
+    """The synthetic generator rounds to bf16 first; the rounding is nearest-even."""
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.0 ** -130, 3.0e38], dtype=np.float32)
+    r = synth.round_bf16(x)
+    t = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(r, t)
+    big = np.random.default_rng(14).standard_normal(100000).astype(np.float32)
+    np.testing.assert_array_equal(synth.round_bf16(big),
+                                  torch.from_numpy(big).to(torch.bfloat16).float().numpy())
