@@ -1,0 +1,444 @@
+#!/usr/bin/env python3
+"""Benchmark of the selective-scan forward on B200 (one JSON line on rank 0).
+
+Default workload: the Mamba-130M-shaped layer (batch 8, d_inner 1536, seqlen 2048,
+d_state 16, bf16 activations, fp32 state, fused causal conv1d width 4 + SiLU,
+softplus delta, z gate). One step = one ssm_selective_scan_fwd call over one
+batch: conv + SiLU, softplus, discretisation, recurrence, readout and gate.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload m130|long|bidir|tiny|decode]
+                  [--impl ours|reference]
+
+Timing: W untimed steps, then K steps bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream; the max over
+ranks is reported. The m130 step streams 201 MB (> 126 MB L2), so no L2 flush is
+inserted between steps. Under torchrun every rank runs its own replica of the
+workload (the path needs no exchange between GPUs): weak scaling.
+
+`--impl reference` times the CPU oracle (double precision, single thread) on a
+bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mamba_selective_scan_sm_b200 import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+SFU_EX2_PER_CLK_PER_SM = 16      # MUFU.EX2 results per clock per SM (measured: see the design doc)
+N_SM = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="m130", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--chunks", type=int, default=0, help="num_chunks passed to the scan (0 = auto)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ bytes --
+
+def algorithmic_bytes(w) -> int:
+    """Compulsory HBM bytes of one step: every input read once, every output written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    if w.name.startswith("decode"):
+        rows = w.batch * w.dim
+        return (rows * w.dstate * 4 * 2          # state read + write
+                + rows * 4 * es * 2              # conv state read + write
+                + rows * es * 3                  # x, dt, z
+                + rows * es                      # y
+                + w.batch * w.dstate * es * 2    # B_t, C_t
+                + w.dim * (w.dstate + 4 + 4) * 4)  # A, D, dt_bias, conv w/b
+    rows = w.batch * w.dim
+    L = w.seqlen
+    act = rows * L * es * 4                       # u (or x), delta, z read; y write
+    bc = w.batch * w.dstate * L * es * 2          # B, C
+    dirs = 2 if w.bidirectional else 1
+    params = w.dim * (w.dstate + 2) * 4 * dirs + (w.dim * (w.conv_width + 1) * 4 if w.conv_width else 0)
+    fstate = rows * w.dstate * 4 * dirs if (w.final_state or w.bidirectional) else 0
+    return act + bc + params + fstate
+
+
+def exp_count(w) -> int:
+    dirs = 2 if w.bidirectional else 1
+    steps = max(w.seqlen, 1) * (w.steps if w.steps else 1)
+    return w.batch * w.dim * steps * w.dstate * dirs
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": rows[0]["max"],
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------- workload --
+
+class ScanWorkload:
+    def __init__(self, w, device, chunks):
+        import torch
+        self.w = w
+        self.torch = torch
+        self.chunks = chunks
+        inp = synth.scan_inputs(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, w.conv_width,
+                                w.bidirectional, seed=0)
+        self.host_inp = inp
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        act = lambda k: torch.from_numpy(inp[k]).to(device).to(tdt)
+        par = lambda k: torch.from_numpy(inp[k]).to(device) if inp.get(k) is not None else None
+        self.t = {k: act(k) for k in ("u", "delta", "z", "B", "C")}
+        self.p = {k: par(k) for k in ("A", "D", "delta_bias", "conv_w", "conv_b", "A_rev", "D_rev",
+                                      "delta_bias_rev")}
+        self.out = torch.empty_like(self.t["u"])
+        shp = (w.batch, w.dim, w.dstate)
+        self.fs = torch.empty(shp, device=device) if (w.final_state or w.bidirectional) else None
+        self.fsr = torch.empty(shp, device=device) if w.bidirectional else None
+        import mamba_selective_scan_sm_b200 as ssm
+        self.ssm = ssm
+        n = ssm.ssm_selective_scan_workspace_size(self.t["u"], self.p["A"],
+                                                  conv_weight=self.p["conv_w"] if w.conv_width else None,
+                                                  A_rev=self.p["A_rev"], num_chunks=chunks)
+        self.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+        self.launches_per_step = 2 if chunks > 1 else 1
+        self.h = None          # pinned host buffers of the end-to-end measurement
+
+    def step(self, t=None):
+        w, p = self.w, self.p
+        t = t or self.t
+        conv = w.conv_width > 0
+        self.ssm.ssm_selective_scan_fwd(
+            t["u"], t["delta"], p["A"], t["B"], t["C"], p["D"], t["z"], p["delta_bias"], True,
+            False, p["conv_w"] if conv else None, p["conv_b"] if conv else None, p["A_rev"],
+            p["D_rev"], p["delta_bias_rev"], out=self.out, num_chunks=self.chunks,
+            workspace=self.ws, final_state=self.fs, final_state_rev=self.fsr)
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.h = {k: v.cpu().pin_memory() for k, v in self.t.items()}
+        self.hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d = sum(v.numel() * v.element_size() for v in self.h.values())
+        self.d2h = self.hout.numel() * self.hout.element_size()
+
+    def e2e_step(self):
+        for k, v in self.h.items():
+            self.t[k].copy_(v, non_blocking=True)
+        self.step()
+        self.hout.copy_(self.out, non_blocking=True)
+
+    def elems(self):
+        return self.w.batch * self.w.dim * self.w.seqlen
+
+
+class DecodeWorkload:
+    """64 successive single-token updates (one step = one token for every row)."""
+
+    def __init__(self, w, device):
+        import torch
+        import mamba_selective_scan_sm_b200 as ssm
+        self.w, self.torch, self.ssm = w, torch, ssm
+        inp = synth.decode_inputs(w.batch, w.dim, w.dstate, w.steps, 4, w.dtype, seed=0)
+        self.host_inp = inp
+        bf = torch.bfloat16
+        self.state = torch.from_numpy(inp["state"]).to(device)
+        self.cs = torch.from_numpy(inp["conv_state"]).to(device).to(bf)
+        self.seq = {k: torch.from_numpy(inp[k]).to(device).to(bf) for k in ("x", "dt", "z", "B", "C")}
+        self.p = {k: torch.from_numpy(inp[k]).to(device) for k in ("A", "D", "dt_bias", "conv_w", "conv_b")}
+        self.out = torch.empty(w.batch, w.dim, dtype=bf, device=device)
+        self.k = 0
+        self.launches_per_step = 1
+        self.h = None
+
+    def step(self):
+        s = self.k % self.w.steps
+        self.k += 1
+        q, p = self.seq, self.p
+        self.ssm.ssm_selective_state_update(self.state, self.cs, q["x"][s], q["dt"][s], p["A"],
+                                            q["B"][s], q["C"][s], p["D"], q["z"][s], p["dt_bias"],
+                                            True, p["conv_w"], p["conv_b"], out=self.out)
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.h = {k: v[0].cpu().pin_memory() for k, v in self.seq.items()}
+        self.hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d = sum(v.numel() * v.element_size() for v in self.h.values())
+        self.d2h = self.hout.numel() * self.hout.element_size()
+
+    def e2e_step(self):
+        s = self.k % self.w.steps
+        for k, v in self.h.items():
+            self.seq[k][s].copy_(v, non_blocking=True)
+        self.step()
+        self.hout.copy_(self.out, non_blocking=True)
+
+    def elems(self):
+        return self.w.batch * self.w.dim
+
+
+# ------------------------------------------------------------ cpu oracle --
+
+def oracle_sample(w, seconds=10.0):
+    """Time the CPU oracle on a bounded sample of the workload; returns (elems/s, desc, cores)."""
+    import oracle
+    if w.name.startswith("decode"):
+        inp = synth.decode_inputs(1, 256, w.dstate, 4, 4, w.dtype, seed=0)
+        t0 = time.perf_counter()
+        n = 0
+        st, cs = inp["state"], inp["conv_state"]
+        while time.perf_counter() - t0 < seconds:
+            for s in range(4):
+                _, st, cs = oracle.state_update(st, cs, inp["x"][s], inp["dt"][s], inp["A"],
+                                                inp["B"][s], inp["C"][s], inp["D"], inp["z"][s],
+                                                inp["dt_bias"], True, inp["conv_w"], inp["conv_b"])
+                n += 256
+        dt = time.perf_counter() - t0
+        return n / dt, f"{n} single-token channel updates (batch 1, d_inner 256) of the decode workload", 1
+    chans_per_call = 16
+    inp = synth.scan_inputs(1, chans_per_call, w.seqlen, w.dstate, w.dtype, w.conv_width,
+                            w.bidirectional, seed=0)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.scan_channels(inp, [(0, d) for d in range(chans_per_call)], conv=w.conv_width > 0,
+                             bidirectional=w.bidirectional)
+        n += chans_per_call * w.seqlen
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    return n / dt, (f"{n // w.seqlen} channels x seqlen {w.seqlen} of the {w.name} workload "
+                    f"({n} elements, {dt:.1f} s)"), 1
+
+
+# -------------------------------------------------------------------- main --
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    steps_v = []
+    for _ in range(args.warmup):
+        oracle_sample(w, seconds=0.5)
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        v, desc, cores = oracle_sample(w, seconds=2.0)
+        steps_v.append(v)
+    wall = time.perf_counter() - t_all
+    value = statistics.median(steps_v)
+    line = {
+        "impl": "reference", "metric": "selective-scan fwd B*D*L elems/s (CPU oracle, fp64)",
+        "value": value, "unit": "elems/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": wall / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": "elems/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    c = {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "seqlen": w.seqlen,
+         "d_state": w.dstate, "conv_width": w.conv_width, "bidirectional": w.bidirectional,
+         "final_state": w.final_state, "parallelism": f"replicas x{args.gpus}"}
+    if w.steps:
+        c["decode_steps_cycled"] = w.steps
+    ab = algorithmic_bytes(w)
+    c["l2"] = ("inputs larger than L2 ({:.0f} MB/step > 126 MB)".format(ab / 1e6)
+               if ab > L2_BYTES else "working set {:.0f} MB/step fits L2: L2-warm".format(ab / 1e6))
+    if args.chunks:
+        c["num_chunks"] = args.chunks
+    return c
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    wl = DecodeWorkload(w, device) if w.name.startswith("decode") else ScanWorkload(w, device, args.chunks)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        wl.step()
+    barrier()
+
+    # per-launch timing of the (single) kernel of a step, for the roofline
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[2 * i].record(stream)
+        wl.step()
+        ev[2 * i + 1].record(stream)
+    t1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms_total = t0.elapsed_time(t1)
+    per_launch = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)]
+    if world > 1:
+        tt = torch.tensor([ms_total], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    elems = wl.elems()
+    value = elems * world / (ms_step * 1e-3)
+
+    # end to end: pinned host inputs -> device -> scan -> device result -> host
+    e2e = None
+    if not args.no_e2e:
+        wl.e2e_setup()
+        for _ in range(3):
+            wl.e2e_step()
+        barrier()
+        k = max(3, min(args.steps, 20))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k):
+            wl.e2e_step()
+        b.record(stream)
+        barrier()
+        ms = a.elapsed_time(b) / k
+        if world > 1:
+            tt = torch.tensor([ms], device=device)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+        e2e = {"value": elems * world / (ms * 1e-3), "unit": "elems/s",
+               "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": ms}
+
+    if rank == 0:
+        hbm_peak, peak_kind = measured_peaks()
+        ab = algorithmic_bytes(w)
+        mean_launch_ms = statistics.mean(per_launch)
+        achieved = ab / (mean_launch_ms * 1e-3) / 1e9
+        sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+        exps = exp_count(w) / (w.steps if w.steps else 1) if w.name.startswith("decode") else exp_count(w)
+        sfu_peak = N_SM * SFU_EX2_PER_CLK_PER_SM * sm_mhz * 1e6
+        sfu_ach = exps / (mean_launch_ms * 1e-3)
+        line = {
+            "metric": "selective-scan fwd B*D*L elems/s and achieved HBM GB/s vs B200 peak (1 GPU)",
+            "value": value, "unit": "elems/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded; value distributions of the Mamba init)",
+            "config": config_of(w, args),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "algorithmic_bytes_per_launch": ab,
+                         "mean_launch_ms": mean_launch_ms},
+            "sfu": {"achieved": sfu_ach, "peak": sfu_peak, "unit": "ex2/s",
+                    "frac": sfu_ach / sfu_peak, "exp2_per_launch": exps,
+                    "peak_kind": f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk x {sm_mhz:.0f} MHz"},
+            "e2e": e2e,
+            "gpu_launches": args.steps * wl.launches_per_step,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            v, desc, cores = oracle_sample(w, seconds=10.0)
+            line["cpu_baseline"] = {"value": v, "unit": "elems/s", "cores": cores,
+                                    "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,176 @@
-"""Mamba selective-scan forward and decode state update for B200 (sm_100a)."""
+"""Mamba selective-scan forward and decode state update for B200 (sm_100a).
+
+A thin binding over the C ABI in include/ssm.h: it takes torch CUDA tensors,
+passes their device pointers and the current stream to libssm_b200.so, and
+allocates the outputs (and the scan's workspace) through torch. Every step of
+the computation runs in the library's kernels; there is no fallback, and a
+missing library raises ``LibraryMissing``.
+
+Functions carry the ABI's names:
+
+* ``ssm_causal_conv1d_fwd(x, w, bias=None, apply_silu=True)``
+* ``ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, ...)``
+* ``ssm_selective_state_update(state, conv_state, x, dt, A, B, C, ...)`` (in place)
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _abi
+from ._abi import LibraryMissing, SSMError, ScanArgs  # noqa: F401
+
+__all__ = ["ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_scan_workspace_size",
+           "ssm_selective_state_update", "ssm_device_error", "LibraryMissing", "SSMError"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return _abi.SSM_F32
+    if t.dtype == torch.bfloat16:
+        return _abi.SSM_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr() if t.numel() else None
+
+
+def _fp32(t, name):
+    if t is not None and t.dtype != _torch().float32:
+        raise TypeError(f"{name} must be float32")
+    return _ptr(t)
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
+               conv_bias, A_rev, D_rev, delta_bias_rev, out, final_state, final_state_rev,
+               num_chunks):
+    batch, dim, seqlen = u.shape
+    a = ScanArgs()
+    a.dtype = _dtype_code(u)
+    a.batch, a.dim, a.seqlen, a.dstate = batch, dim, seqlen, A.shape[1]
+    a.u, a.delta, a.B, a.C, a.z = _ptr(u), _ptr(delta), _ptr(B), _ptr(C), _ptr(z)
+    a.A, a.D, a.delta_bias = _fp32(A, "A"), _fp32(D, "D"), _fp32(delta_bias, "delta_bias")
+    a.delta_softplus, a.reverse = int(bool(delta_softplus)), int(bool(reverse))
+    a.conv_weight, a.conv_bias = _fp32(conv_weight, "conv_weight"), _fp32(conv_bias, "conv_bias")
+    a.conv_width = conv_weight.shape[1] if conv_weight is not None else 0
+    a.A_rev, a.D_rev = _fp32(A_rev, "A_rev"), _fp32(D_rev, "D_rev")
+    a.delta_bias_rev = _fp32(delta_bias_rev, "delta_bias_rev")
+    a.out = _ptr(out)
+    a.final_state, a.final_state_rev = _ptr(final_state), _ptr(final_state_rev)
+    a.num_chunks = int(num_chunks)
+    return a
+
+
+def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num_chunks=0,
+                                      reverse=False):
+    """Workspace bytes ssm_selective_scan_fwd needs for these shapes (host-only query)."""
+    lib = _abi.load()
+    a = ScanArgs()
+    a.dtype = _dtype_code(u)
+    a.batch, a.dim, a.seqlen = u.shape
+    a.dstate = A.shape[1]
+    a.reverse = int(bool(reverse))
+    a.A_rev = 1 if A_rev is not None else None
+    a.conv_weight = 1 if conv_weight is not None else None
+    a.conv_width = conv_weight.shape[1] if conv_weight is not None else 0
+    a.num_chunks = int(num_chunks)
+    n = ctypes.c_size_t()
+    _abi.check(lib, lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                           delta_softplus=True, reverse=False, conv_weight=None, conv_bias=None,
+                           A_rev=None, D_rev=None, delta_bias_rev=None, *, out=None,
+                           return_final_state=False, final_state=None, final_state_rev=None,
+                           num_chunks=0, workspace=None, stream=None):
+    """Selective-scan forward (see include/ssm.h). Layouts: u, delta, z (batch, dim, seqlen);
+    B, C (batch, dstate, seqlen); A (dim, dstate) fp32. With ``conv_weight`` (dim, width), ``u``
+    is the pre-conv x. With ``A_rev`` the result is the bidirectional sum.
+
+    ``final_state`` / ``final_state_rev`` may be given as preallocated fp32 outputs
+    (batch, dim, dstate); they are written whenever given.
+    Returns ``out`` or ``(out, final_state[, final_state_rev])``.
+    """
+    torch = _torch()
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty_like(u)
+    fs, fsr = final_state, final_state_rev
+    if return_final_state:
+        shp = (u.shape[0], u.shape[1], A.shape[1])
+        if fs is None:
+            fs = torch.empty(shp, dtype=torch.float32, device=u.device)
+        if A_rev is not None and fsr is None:
+            fsr = torch.empty(shp, dtype=torch.float32, device=u.device)
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
+                   conv_bias, A_rev, D_rev, delta_bias_rev, out, fs, fsr, num_chunks)
+    n = ctypes.c_size_t()
+    _abi.check(lib, lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    if n.value:
+        if workspace is None or workspace.numel() < n.value:
+            workspace = torch.empty(n.value, dtype=torch.uint8, device=u.device)
+        a.workspace, a.workspace_bytes = _ptr(workspace), n.value
+    _abi.check(lib, lib.ssm_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
+    if not return_final_state:
+        return out
+    return (out, fs, fsr) if A_rev is not None else (out, fs)
+
+
+def ssm_causal_conv1d_fwd(x, w, bias=None, apply_silu=True, *, out=None, stream=None):
+    """Causal depthwise conv1d (+ SiLU). x (batch, dim, seqlen); w (dim, width) fp32."""
+    torch = _torch()
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty_like(x)
+    batch, dim, seqlen = x.shape
+    _abi.check(lib, lib.ssm_causal_conv1d_fwd(_ptr(x), _fp32(w, "w"), _fp32(bias, "bias"),
+                                              _ptr(out), batch, dim, seqlen, w.shape[1],
+                                              int(bool(apply_silu)), _dtype_code(x),
+                                              _stream(stream)))
+    return out
+
+
+def ssm_selective_state_update(state, conv_state, x, dt, A, B, C, D=None, z=None, dt_bias=None,
+                               dt_softplus=True, conv_weight=None, conv_bias=None, *, out=None,
+                               stream=None):
+    """One decode step, in place on ``state`` (batch, dim, dstate) fp32 and ``conv_state``
+    (batch, dim, width). x, dt, z (batch, dim); B, C (batch, dstate). Returns y (batch, dim)."""
+    torch = _torch()
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty_like(x)
+    batch, dim, dstate = state.shape
+    width = conv_weight.shape[1] if conv_weight is not None else 0
+    _abi.check(lib, lib.ssm_selective_state_update(
+        _fp32(state, "state"), _ptr(conv_state), _ptr(x), _ptr(dt), _fp32(A, "A"), _ptr(B),
+        _ptr(C), _fp32(D, "D"), _ptr(z), _fp32(dt_bias, "dt_bias"), int(bool(dt_softplus)),
+        _fp32(conv_weight, "conv_weight"), _fp32(conv_bias, "conv_bias"), width, _ptr(out),
+        batch, dim, dstate, _dtype_code(x), _stream(stream)))
+    return out
+
+
+def ssm_device_error(stream=None) -> int:
+    """Read and clear the library's device error word (synchronises the stream)."""
+    lib = _abi.load()
+    code = ctypes.c_int32()
+    _abi.check(lib, lib.ssm_device_error(ctypes.byref(code), _stream(stream)))
+    return code.value

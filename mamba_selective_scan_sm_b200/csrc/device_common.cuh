@@ -1,0 +1,129 @@
+// Device-side helpers shared by the sm_100a kernels: element conversion, the
+// exponentials used by the scan, and TMA / mbarrier primitives with bounded waits.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// ---------------------------------------------------------------- elements --
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float* p) { return *p; }
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p) {
+        return __bfloat162float(*p);
+    }
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) {
+        return __float2bfloat16_rn(v);
+    }
+};
+
+// ------------------------------------------------------------------- math --
+
+// 2^x on the SFU (one MUFU.EX2). Inputs far below -126 flush to 0, which is the
+// limit the recurrence wants for a fully decayed state.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// softplus(x) = log(1 + e^x). Above 20 the correction log1p(e^-x) < 2.1e-9 is far
+// below fp32 resolution of x, so x itself is returned.
+__device__ __forceinline__ float softplus(float x) {
+    return x > 20.f ? x : log1pf(__expf(x));
+}
+
+// silu(v) = v * sigmoid(v) = v / (1 + e^-v); tends to 0 for v -> -inf.
+__device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
+
+// ------------------------------------------------------- shared / barriers --
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait budget of a single mbarrier wait. A TMA tile lands in microseconds; a wait
+// that lasts this long means the copy will not complete.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+
+// Device-side error word (read and cleared by ssm_device_error()). Defined here:
+// exactly one translation unit (kernels.cu) includes the device headers.
+__device__ int g_device_error = 0;
+
+// Bounded wait on an mbarrier phase. Returns false (and records the error) when
+// the budget runs out; the caller must then leave the kernel uniformly.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicExch(&g_device_error, 1);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------- TMA --
+
+// 3-D tiled TMA load into this CTA's shared memory, completing on `bar`.
+// The innermost coordinate c0 times the element size must be a multiple of 16 B.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+}  // namespace ssm

@@ -1,0 +1,105 @@
+// Device code of the library: one translation unit holding every kernel, the
+// device error word and the host launchers that pick a template variant.
+#include "conv_kernel.cuh"
+#include "decode_kernel.cuh"
+#include "launch.h"
+#include "scan_kernel.cuh"
+
+namespace ssm {
+
+namespace {
+
+template <typename T, int NP, int S>
+ScanVariant variant_of() {
+    using Cfg = ScanCfg<T, NP, S>;
+    return ScanVariant{(int)sizeof(T), NP, S, Cfg::G, Cfg::TT, Cfg::HALO, Cfg::SMEM};
+}
+
+template <typename T, int NP, int S, bool TMA, bool SUM>
+cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
+    using Cfg = ScanCfg<T, NP, S>;
+    auto* k = scan_fwd_kernel<T, NP, S, TMA, SUM>;
+    static const cudaError_t attr =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kScanThreads, Cfg::SMEM, st>>>(maps, p);
+    return cudaGetLastError();
+}
+
+template <typename T, int NP, int S>
+cudaError_t launch_t(bool tma, bool sum, const ScanMaps& maps, const ScanParams& p, dim3 grid,
+                     cudaStream_t st) {
+    if (tma) return sum ? launch_one<T, NP, S, true, true>(maps, p, grid, st)
+                        : launch_one<T, NP, S, true, false>(maps, p, grid, st);
+    return sum ? launch_one<T, NP, S, false, true>(maps, p, grid, st)
+               : launch_one<T, NP, S, false, false>(maps, p, grid, st);
+}
+
+}  // namespace
+
+#define SSM_SCAN_VARIANTS(X) \
+    X(4, 4)                  \
+    X(2, 8)                  \
+    X(2, 4)                  \
+    X(1, 4)
+
+bool scan_variant(int es, int np, int s, ScanVariant* v) {
+#define X(NP_, S_)                                                          \
+    if (np == NP_ && s == S_) {                                             \
+        *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_>()                 \
+                     : variant_of<float, NP_, S_>();                        \
+        return es == 2 || es == 4;                                          \
+    }
+    SSM_SCAN_VARIANTS(X)
+#undef X
+    return false;
+}
+
+cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
+                        const ScanParams& p, dim3 grid, cudaStream_t st) {
+#define X(NP_, S_)                                                                    \
+    if (v.np == NP_ && v.s == S_)                                                     \
+        return v.elem_size == 2 ? launch_t<__nv_bfloat16, NP_, S_>(tma, sum, maps, p, grid, st) \
+                                : launch_t<float, NP_, S_>(tma, sum, maps, p, grid, st);
+    SSM_SCAN_VARIANTS(X)
+#undef X
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) {
+    const int64_t per_row = (p.seqlen + 7) / 8;
+    const int64_t threads = p.rows * per_row;
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (es == 2) {
+        if (vec) conv1d_kernel<__nv_bfloat16, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else conv1d_kernel<__nv_bfloat16, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+    } else {
+        if (vec) conv1d_kernel<float, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else conv1d_kernel<float, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_t st) {
+    // 4 lanes x 4 states covers dstate <= 16
+    const int64_t threads = p.rows * 4;
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    (void)dstate;
+    if (es == 2) decode_kernel<__nv_bfloat16, 4, 4><<<(unsigned)blocks, 256, 0, st>>>(p);
+    else decode_kernel<float, 4, 4><<<(unsigned)blocks, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t read_device_error(int* code, cudaStream_t st) {
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_device_error, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(st);
+}
+
+}  // namespace ssm

@@ -1,0 +1,34 @@
+// Host-side launchers of the device kernels (defined in kernels.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "scan_params.h"
+
+namespace ssm {
+
+// Static shape of one scan-kernel variant.
+struct ScanVariant {
+    int elem_size;      // 2 (bf16) or 4 (fp32)
+    int np;             // states per lane
+    int s;              // lanes per channel
+    int channels;       // channels per CTA (128 / s)
+    int tile;           // time steps per tile (128 bytes of elements)
+    int halo;           // conv history elements fetched with a tile
+    int smem_bytes;     // dynamic shared memory per CTA
+};
+
+// Returns false if (elem_size, np, s) has no compiled kernel.
+bool scan_variant(int elem_size, int np, int s, ScanVariant* v);
+
+cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, const ScanMaps& maps,
+                        const ScanParams& p, dim3 grid, cudaStream_t stream);
+
+cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream_t stream);
+
+cudaError_t launch_decode(int elem_size, int dstate, const DecodeParams& p, cudaStream_t stream);
+
+// Read and clear the device error word (synchronises `stream`).
+cudaError_t read_device_error(int* code, cudaStream_t stream);
+
+}  // namespace ssm

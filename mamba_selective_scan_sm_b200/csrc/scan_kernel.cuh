@@ -1,0 +1,479 @@
+// Selective-scan forward kernel for sm_100a.
+//
+// Work split. A CTA of 128 threads owns G = 128/S channels of one batch row and
+// walks the sequence in tiles of TT = 32 time steps.
+// The S lanes of a channel each keep NP = NS/S of the (padded) NS states in
+// registers, so one channel's recurrence is spread over S lanes with no carry
+// between them (A is diagonal: the states never interact).
+//
+// Per tile:
+//   1. TMA brings the raw tiles (u or the pre-conv x with a 16-byte halo, dt, z,
+//      B, C) into a 2-stage shared-memory ring; B and C are shared by the CTA's
+//      channels (all channels of a batch row read the same B_t, C_t).
+//   2. Prologue, once per (channel, t): conv + SiLU, delta = softplus(dt + bias),
+//      delta*u, D*u and silu(z) -> fp32 staging buffers; B and C are transposed to
+//      [t][n] fp32 so each lane reads its NP states with one vector load.
+//   3. Scan: per (t, state) one ex2 on the SFU, then h = dA*h + delta*u*B and the
+//      lane's partial C.h. Every 16 steps a butterfly transpose-reduce over the S
+//      lanes leaves each lane owning 16/S consecutive outputs, which it gates and
+//      stores with one vector store.
+//
+// Two-pass chunk carry (paperlayer.ai summary of arXiv 2603.09555, §3 Method,
+// "Chunked recurrence"): with nchunks > 1, a SUMMARY launch scans every chunk but
+// the last from a zero state and writes (prod dA, h_end) per state; the output
+// launch starts chunk k from the carry H_k = P_{k-1} H_{k-1} + S_{k-1}.
+#pragma once
+
+#include "device_common.cuh"
+#include "scan_params.h"
+
+namespace ssm {
+
+constexpr int kScanThreads = 128;
+
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+template <typename T, int NP, int S>
+struct ScanCfg {
+    static constexpr int NT = kScanThreads;
+    static constexpr int G = NT / S;          // channels per CTA
+    static constexpr int NS = NP * S;         // padded state count
+    static constexpr int ES = sizeof(T);
+    static constexpr int TT = 32;             // tile length (time steps)
+    static constexpr int ROWB = TT * ES;      // bytes of one tile row: 64 (bf16) / 128 (fp32)
+    static constexpr int SWZ = ROWB == 128 ? 7 : 3;   // TMA 128-B / 64-B swizzle mask
+    static constexpr int HALO = 16 / ES;      // conv history, one 16-B TMA granule
+    static constexpr int NSTAGE = 2;
+    static constexpr int R = 16 / S;          // outputs owned per lane per 16-step block
+    // raw stage (bytes from the 1024-aligned stage base)
+    static constexpr int RAW_B = 0;                                   // [NS][TT], swizzled
+    static constexpr int RAW_C = align_up(NS * ROWB, 1024);           // [NS][TT], swizzled
+    static constexpr int RAW_X = align_up(RAW_C + NS * ROWB, 128);    // [G][TT(+HALO)]
+    static constexpr int X_PITCH_MAX = (TT + HALO) * ES;
+    static constexpr int RAW_DT = align_up(RAW_X + G * X_PITCH_MAX, 128);
+    static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, 128);
+    static constexpr int STAGE = align_up(RAW_Z + G * ROWB, 1024);
+    // fp32 staging
+    static constexpr int P_PITCH = TT * 8 + 8;            // float2 {delta, delta*u}
+    static constexpr int E_PITCH = TT * 8 + 16;           // float2 {D*u, silu(z)}
+    static constexpr int OFF_P = NSTAGE * STAGE;
+    static constexpr int OFF_E = OFF_P + G * P_PITCH;
+    static constexpr int OFF_BT = align_up(OFF_E + G * E_PITCH, 16);
+    static constexpr int OFF_CT = OFF_BT + TT * NS * 4;
+    static constexpr int OFF_PAR = OFF_CT + TT * NS * 4;  // 8 floats per channel
+    static constexpr int OFF_BAR = align_up(OFF_PAR + G * 32, 8);
+    static constexpr int BYTES = OFF_BAR + NSTAGE * 8;
+    static constexpr int SMEM = BYTES + 1024;             // slack for 1024-B alignment
+    static_assert(TT % 16 == 0, "tile must hold whole 16-step blocks");
+    static_assert(NS <= 16, "at most 16 states");
+};
+
+// Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 128-B
+// and 64-B swizzles XOR address bits [4, 4+k) with bits [7, 7+k) (k = 3 or 2) of
+// the offset from a 1024-byte aligned tile base; SWZ is the k-bit mask.
+template <int ROWB, int SWZ>
+__device__ __forceinline__ int swz(int row, int byte_in_row) {
+    const int off = row * ROWB + byte_in_row;
+    return off ^ (((off >> 7) & SWZ) << 4);
+}
+
+template <typename T, int NP, int S, bool USE_TMA, bool SUMMARY>
+__global__ void __launch_bounds__(kScanThreads)
+scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
+    using Cfg = ScanCfg<T, NP, S>;
+    using E = Elem<T>;
+    constexpr int G = Cfg::G, NS = Cfg::NS, TT = Cfg::TT, HALO = Cfg::HALO, R = Cfg::R;
+    constexpr int ROWB = Cfg::ROWB, SWZ = Cfg::SWZ;
+    constexpr int NSTAGE = Cfg::NSTAGE;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float2* Pbuf = reinterpret_cast<float2*>(smem + Cfg::OFF_P);
+    float2* Ebuf = reinterpret_cast<float2*>(smem + Cfg::OFF_E);
+    float* Bt = reinterpret_cast<float*>(smem + Cfg::OFF_BT);
+    float* Ct = reinterpret_cast<float*>(smem + Cfg::OFF_CT);
+    float* par = reinterpret_cast<float*>(smem + Cfg::OFF_PAR);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int c = tid / S;          // channel slot in the CTA
+    const int j = tid % S;          // state group of this lane
+    const int b = blockIdx.y;
+    const int d0 = blockIdx.x * G;
+    const int d = d0 + c;
+    const bool dvalid = d < p.dim;
+    const int L = p.seqlen;
+    const int chunk = blockIdx.z;
+    const int cs = chunk * p.chunk_len;                    // first scan position
+    const int ce = min(cs + p.chunk_len, L);               // one past the last
+    const int ntl = (ce - cs + TT - 1) / TT;               // tiles per direction
+    const int ndir = p.mode == 2 ? 2 : 1;
+    const int nt = ntl * ndir;
+    const bool has_z = !SUMMARY && p.z != nullptr;
+    const bool conv = p.conv_w != nullptr;
+    const int xpitch = conv ? Cfg::X_PITCH_MAX : TT * (int)sizeof(T);
+    const int64_t row = (int64_t)b * p.dim + d;           // (b, d) row index
+
+    auto tile_rev = [&](int f) { return p.mode == 1 || (p.mode == 2 && f >= ntl); };
+    // time of the first element of flat tile f
+    auto tile_l0 = [&](int f) {
+        const int jt = f % ntl;
+        const int i0 = cs + jt * TT;
+        return tile_rev(f) ? L - i0 - TT : i0;
+    };
+
+    if (USE_TMA && tid == 0) {
+        for (int s = 0; s < NSTAGE; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        prefetch_tensormap(&maps.x);
+        prefetch_tensormap(&maps.dt);
+        prefetch_tensormap(&maps.B);
+        prefetch_tensormap(&maps.C);
+        if (has_z) prefetch_tensormap(&maps.z);
+    }
+
+    auto issue = [&](int f) {   // one thread: TMA loads of flat tile f
+        uint8_t* st = smem + (f % NSTAGE) * Cfg::STAGE;
+        const int l0 = tile_l0(f);
+        const bool rv = tile_rev(f);
+        const uint32_t xbytes = G * xpitch;
+        uint32_t bytes = 2u * NS * ROWB + xbytes + G * ROWB + (has_z ? G * ROWB : 0u);
+        mbar_arrive_expect_tx(&bars[f % NSTAGE], bytes);
+        tma_load_3d(st + Cfg::RAW_B, &maps.B, &bars[f % NSTAGE], l0, 0, b);
+        tma_load_3d(st + Cfg::RAW_C, &maps.C, &bars[f % NSTAGE], l0, 0, b);
+        tma_load_3d(st + Cfg::RAW_X, &maps.x, &bars[f % NSTAGE], (conv && !rv) ? l0 - HALO : l0,
+                    d0, b);
+        tma_load_3d(st + Cfg::RAW_DT, &maps.dt, &bars[f % NSTAGE], l0, d0, b);
+        if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, &bars[f % NSTAGE], l0, d0, b);
+    };
+
+    // Plain-load fallback (any alignment): fills stage 0 with the same layout.
+    auto load_plain = [&](int f) {
+        uint8_t* st = smem;
+        const int l0 = tile_l0(f);
+        const bool rv = tile_rev(f);
+        const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
+        const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
+        for (int e = tid; e < NS * TT; e += kScanThreads) {
+            const int n = e / TT, col = e % TT, t = l0 + col;
+            const bool ok = n < p.dstate && t >= 0 && t < L;
+            const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
+            *reinterpret_cast<T*>(st + Cfg::RAW_B + off) = ok ? gB[(int64_t)n * L + t] : T(0.f);
+            *reinterpret_cast<T*>(st + Cfg::RAW_C + off) = ok ? gC[(int64_t)n * L + t] : T(0.f);
+        }
+        const int xw = xpitch / (int)sizeof(T);
+        const int xs = (conv && !rv) ? l0 - HALO : l0;
+        for (int e = tid; e < G * xw; e += kScanThreads) {
+            const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
+            const bool ok = dd < p.dim && t >= 0 && t < L;
+            const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
+            reinterpret_cast<T*>(st + Cfg::RAW_X + r * xpitch)[col] =
+                ok ? static_cast<const T*>(p.u)[gi] : T(0.f);
+        }
+        for (int e = tid; e < G * TT; e += kScanThreads) {
+            const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
+            const bool ok = dd < p.dim && t >= 0 && t < L;
+            const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
+            reinterpret_cast<T*>(st + Cfg::RAW_DT)[r * TT + col] =
+                ok ? static_cast<const T*>(p.delta)[gi] : T(0.f);
+            if (has_z)
+                reinterpret_cast<T*>(st + Cfg::RAW_Z)[r * TT + col] =
+                    ok ? static_cast<const T*>(p.z)[gi] : T(0.f);
+        }
+    };
+
+    // Per-direction channel parameters -> smem (8 floats per channel slot).
+    auto load_params = [&](int dir) {
+        for (int e = tid; e < G; e += kScanThreads) {
+            const int dd = d0 + e;
+            float* q = par + e * 8;
+            const bool ok = dd < p.dim;
+            // conv taps right-aligned: q[3] meets the newest input
+            for (int k = 0; k < 4; ++k) {
+                const int kk = k - (4 - p.conv_width);
+                q[k] = (ok && conv && kk >= 0) ? p.conv_w[(int64_t)dd * p.conv_width + kk] : 0.f;
+            }
+            q[4] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
+            q[5] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
+            q[6] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
+            q[7] = 0.f;
+        }
+    };
+
+    float h[NP], a2[NP], pr[NP];
+    auto load_A = [&](int dir) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const int n = j * NP + k;
+            a2[k] = (dvalid && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
+        }
+    };
+    // Initial state of this chunk: carry over the summaries of earlier chunks.
+    auto init_state = [&]() {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) { h[k] = 0.f; pr[k] = 1.f; }
+        if (!SUMMARY && chunk > 0 && dvalid) {
+            const int64_t stride = (int64_t)p.batch * p.dim * NS;
+            for (int k2 = 0; k2 < chunk; ++k2) {
+                const float2* sm = p.summary + k2 * stride + row * NS + j * NP;
+#pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    const float2 ps = sm[k];
+                    h[k] = fmaf(ps.x, h[k], ps.y);
+                }
+            }
+        }
+    };
+
+    auto prologue = [&](int f, const uint8_t* st) {
+        const bool rv = tile_rev(f);
+        const int xoff = (conv && !rv) ? HALO : 0;
+        // B, C: swizzled [n][t] (input dtype) -> [t][n] fp32
+        for (int e = tid; e < NS * TT; e += kScanThreads) {
+            const int n = e % NS, tt = e / NS;
+            const int off = swz<ROWB, SWZ>(n, tt * (int)sizeof(T));
+            Bt[tt * NS + n] = E::to_f(*reinterpret_cast<const T*>(st + Cfg::RAW_B + off));
+            Ct[tt * NS + n] = E::to_f(*reinterpret_cast<const T*>(st + Cfg::RAW_C + off));
+        }
+        // per (channel, t) quantities; a warp walks one channel row, lanes along t
+        for (int idx = warp; idx < G * (TT / 32); idx += kScanThreads / 32) {
+            const int r = idx / (TT / 32);
+            const int tt = (idx % (TT / 32)) * 32 + lane;
+            const T* xr = reinterpret_cast<const T*>(st + Cfg::RAW_X + r * xpitch);
+            const float* q = par + r * 8;
+            float u;
+            if (conv) {
+                float acc = q[4];
+                if (!rv) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc = fmaf(q[k], E::to_f(xr[xoff + tt - 3 + k]), acc);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc = fmaf(q[k], E::to_f(xr[tt + 3 - k]), acc);
+                }
+                u = silu(acc);
+            } else {
+                u = E::to_f(xr[tt]);
+            }
+            float dl = E::to_f(reinterpret_cast<const T*>(st + Cfg::RAW_DT)[r * TT + tt]) + q[5];
+            if (p.softplus) dl = softplus(dl);
+            reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(Pbuf) + r * Cfg::P_PITCH)[tt] =
+                make_float2(dl, dl * u);
+            if (!SUMMARY) {
+                const float g =
+                    has_z ? silu(E::to_f(reinterpret_cast<const T*>(st + Cfg::RAW_Z)[r * TT + tt]))
+                          : 1.f;
+                reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(Ebuf) + r * Cfg::E_PITCH)[tt] =
+                    make_float2(q[6] * u, g);
+            }
+        }
+    };
+
+    const float2* Prow = reinterpret_cast<const float2*>(reinterpret_cast<uint8_t*>(Pbuf) +
+                                                          c * Cfg::P_PITCH);
+    const float2* Erow = reinterpret_cast<const float2*>(reinterpret_cast<uint8_t*>(Ebuf) +
+                                                          c * Cfg::E_PITCH);
+
+    auto scan_tile = [&](int f) {
+        const bool rv = tile_rev(f);
+        const int dir = (p.mode == 2 && f >= ntl) ? 1 : 0;
+        const int jt = f % ntl;
+        const int i0 = cs + jt * TT;
+        const int nvalid = min(TT, ce - i0);
+        const int l0 = rv ? L - i0 - TT : i0;
+#pragma unroll 1
+        for (int blk = 0; blk < TT / 16; ++blk) {
+            if (blk * 16 >= nvalid) break;
+            float acc[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int ii = blk * 16 + q;
+                const int tt = rv ? TT - 1 - ii : ii;
+                acc[q] = 0.f;
+                if (ii < nvalid) {
+                    const float2 pd = Prow[tt];
+                    float bv[NP], cv[NP];
+                    if constexpr (NP == 4) {
+                        const float4 b4 = *reinterpret_cast<const float4*>(Bt + tt * NS + j * 4);
+                        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+                        if (!SUMMARY) {
+                            const float4 c4 = *reinterpret_cast<const float4*>(Ct + tt * NS + j * 4);
+                            cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+                        }
+                    } else if constexpr (NP == 2) {
+                        const float2 b2 = *reinterpret_cast<const float2*>(Bt + tt * NS + j * 2);
+                        bv[0] = b2.x; bv[1] = b2.y;
+                        if (!SUMMARY) {
+                            const float2 c2 = *reinterpret_cast<const float2*>(Ct + tt * NS + j * 2);
+                            cv[0] = c2.x; cv[1] = c2.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < NP; ++k) {
+                            bv[k] = Bt[tt * NS + j * NP + k];
+                            if (!SUMMARY) cv[k] = Ct[tt * NS + j * NP + k];
+                        }
+                    }
+                    float a = 0.f;
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        const float dA = ex2(pd.x * a2[k]);
+                        h[k] = fmaf(dA, h[k], pd.y * bv[k]);
+                        if (SUMMARY) pr[k] *= dA;
+                        else a = fmaf(cv[k], h[k], a);
+                    }
+                    acc[q] = a;
+                }
+            }
+            if (SUMMARY) continue;
+            // butterfly transpose-reduce over the S lanes of the channel:
+            // afterwards lane j holds the sums for block positions [j*R, j*R + R)
+            int len = 16;
+#pragma unroll
+            for (int m = S / 2; m >= 1; m >>= 1) {
+                const int half = len >> 1;
+                const bool upper = (j & m) != 0;
+#pragma unroll
+                for (int i = 0; i < half; ++i) {
+                    const float send = upper ? acc[i] : acc[i + half];
+                    const float keep = upper ? acc[i + half] : acc[i];
+                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+                len = half;
+            }
+            // epilogue: gate, skip term, (bidirectional partial), store R outputs
+            const int pos0 = blk * 16 + j * R;             // first owned position in tile
+            float yv[R];
+            int tmin;                                      // smallest time among them
+#pragma unroll
+            for (int m = 0; m < R; ++m) {
+                const int ii = pos0 + m;
+                const int tt = rv ? TT - 1 - ii : ii;
+                const float2 e = Erow[tt];
+                yv[m] = (acc[m] + e.x) * e.y;
+            }
+            tmin = rv ? l0 + TT - 1 - (pos0 + R - 1) : l0 + pos0;
+            const int nown = max(0, min(R, nvalid - pos0));
+            if (dvalid && nown > 0) {
+                // time-ascending order
+                float ya[R];
+#pragma unroll
+                for (int m = 0; m < R; ++m) ya[m] = rv ? yv[R - 1 - m] : yv[m];
+                // valid ascending index range: forward [0, nown); reverse [R - nown, R)
+                const int mlo = rv ? R - nown : 0;
+                const int mhi = rv ? R : nown;
+                const int64_t gbase = row * L + tmin;
+                if (p.mode == 2 && dir == 1) {
+#pragma unroll
+                    for (int m = 0; m < R; ++m)
+                        if (m >= mlo && m < mhi) ya[m] += p.partial[gbase + m];
+                }
+                if (p.mode == 2 && dir == 0) {
+#pragma unroll
+                    for (int m = 0; m < R; ++m)
+                        if (m >= mlo && m < mhi) p.partial[gbase + m] = ya[m];
+                } else {
+                    T* out = static_cast<T*>(p.out) + gbase;
+                    const bool full = (mlo == 0 && mhi == R) && p.vec_store;
+                    if (full && R * sizeof(T) == 16) {
+                        if constexpr (sizeof(T) == 4) {
+                            *reinterpret_cast<float4*>(out) = make_float4(ya[0], ya[1 % R], ya[2 % R], ya[3 % R]);
+                        } else {
+                            uint4 v;
+                            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                __nv_bfloat162 t2 = __floats2bfloat162_rn(ya[(2 * m) % R], ya[(2 * m + 1) % R]);
+                                w[m] = *reinterpret_cast<uint32_t*>(&t2);
+                            }
+                            *reinterpret_cast<uint4*>(out) = v;
+                        }
+                    } else if (full && R * sizeof(T) == 8) {
+                        if constexpr (sizeof(T) == 4) {
+                            *reinterpret_cast<float2*>(out) = make_float2(ya[0], ya[1 % R]);
+                        } else {
+                            __nv_bfloat162 t0 = __floats2bfloat162_rn(ya[0], ya[1 % R]);
+                            __nv_bfloat162 t1 = __floats2bfloat162_rn(ya[2 % R], ya[3 % R]);
+                            uint2 v;
+                            v.x = *reinterpret_cast<uint32_t*>(&t0);
+                            v.y = *reinterpret_cast<uint32_t*>(&t1);
+                            *reinterpret_cast<uint2*>(out) = v;
+                        }
+                    } else if (full && R * sizeof(T) == 4 && sizeof(T) == 2) {
+                        *reinterpret_cast<__nv_bfloat162*>(out) =
+                            __floats2bfloat162_rn(ya[0], ya[1 % R]);
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < R; ++m)
+                            if (m >= mlo && m < mhi) out[m] = E::from_f(ya[m]);
+                    }
+                }
+            }
+        }
+    };
+
+    auto finish_direction = [&](int dir) {
+        if (!dvalid) return;
+        if (SUMMARY) {
+            float2* sm = p.summary + (int64_t)chunk * p.batch * p.dim * NS + row * NS + j * NP;
+#pragma unroll
+            for (int k = 0; k < NP; ++k) sm[k] = make_float2(pr[k], h[k]);
+        } else if (chunk == p.nchunks - 1 && p.final_state[dir]) {
+            float* fs = p.final_state[dir] + row * p.dstate;
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = j * NP + k;
+                if (n < p.dstate) fs[n] = h[k];
+            }
+        }
+    };
+
+    // ------------------------------------------------------------- main loop --
+    load_params(0);
+    load_A(0);
+    init_state();
+    if (USE_TMA) {
+        __syncthreads();   // barrier init visible before any wait
+        if (tid == 0)
+            for (int f = 0; f < min(NSTAGE, nt); ++f) issue(f);
+    }
+    __syncthreads();
+
+    for (int f = 0; f < nt; ++f) {
+        if (p.mode == 2 && f == ntl) {       // second direction of the bidirectional sum
+            finish_direction(0);
+            __syncthreads();                 // params of direction 0 no longer read
+            load_params(1);
+            load_A(1);
+#pragma unroll
+            for (int k = 0; k < NP; ++k) { h[k] = 0.f; pr[k] = 1.f; }
+            __syncthreads();
+        }
+        bool ok = true;
+        const uint8_t* st;
+        if (USE_TMA) {
+            ok = mbar_wait_bounded(&bars[f % NSTAGE], (f / NSTAGE) & 1);
+            st = smem + (f % NSTAGE) * Cfg::STAGE;
+        } else {
+            load_plain(f);
+            __syncthreads();
+            st = smem;
+        }
+        prologue(f, st);
+        if (__syncthreads_or(!ok)) {
+            // a tile never landed: drain what is still in flight (bounded), leave
+            if (USE_TMA && tid == 0)
+                for (int g2 = f; g2 < min(f + NSTAGE, nt); ++g2)
+                    mbar_wait_bounded(&bars[g2 % NSTAGE], (g2 / NSTAGE) & 1);
+            return;
+        }
+        if (USE_TMA && tid == 0 && f + NSTAGE < nt) issue(f + NSTAGE);
+        scan_tile(f);
+        __syncthreads();
+    }
+    finish_direction(p.mode == 2 ? 1 : 0);
+}
+
+}  // namespace ssm

@@ -1,0 +1,72 @@
+// Launch parameters of the kernels (host and device view).
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// TMA descriptors of the streamed tensors (unused by the plain-load variant).
+struct ScanMaps {
+    CUtensorMap x;    // u or pre-conv x: dims (L, D, batch), box (TT [+halo], G, 1)
+    CUtensorMap dt;   // delta:           dims (L, D, batch), box (TT, G, 1)
+    CUtensorMap z;    // gate input:      dims (L, D, batch), box (TT, G, 1)
+    CUtensorMap B;    // dims (L, N, batch), box (TT, NS, 1), 128-byte swizzle
+    CUtensorMap C;    // dims (L, N, batch), box (TT, NS, 1), 128-byte swizzle
+};
+
+struct ScanParams {
+    int batch, dim, seqlen, dstate;
+    const void* u;
+    const void* delta;
+    const void* z;          // nullptr: no gate
+    const void* Bm;
+    const void* Cm;
+    const float* A[2];      // per direction (index 1 only for the bidirectional sum)
+    const float* Dv[2];
+    const float* dbias[2];
+    const float* conv_w;    // nullptr: no fused conv
+    const float* conv_b;
+    int conv_width;
+    int softplus;
+    int mode;               // 0 forward, 1 reverse, 2 bidirectional sum
+    void* out;
+    float* partial;         // bidirectional: fp32 buffer for the first direction
+    float* final_state[2];
+    int chunk_len;          // scan positions per chunk (multiple of the tile length)
+    int nchunks;
+    float2* summary;        // two-pass: [nchunks-1][batch*dim][NS] {prod dA, h_end}
+    int vec_store;          // rows are 16-byte aligned: vector stores allowed
+};
+
+// Standalone causal conv1d.
+struct ConvParams {
+    const void* x;
+    const float* w;
+    const float* bias;
+    void* out;
+    int64_t rows;      // batch * dim
+    int dim, seqlen, width, silu;
+};
+
+// Single-token state update.
+struct DecodeParams {
+    float* state;
+    void* conv_state;
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* Bt;
+    const void* Ct;
+    const float* D;
+    const void* z;
+    const float* dt_bias;
+    const float* conv_w;
+    const float* conv_b;
+    void* out;
+    int64_t rows;       // batch * dim
+    int dim, dstate, conv_width, softplus;
+    int vec;            // dstate == 16 and state / A rows 16-byte aligned
+};
+
+}  // namespace ssm

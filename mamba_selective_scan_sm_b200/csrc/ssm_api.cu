@@ -1,0 +1,415 @@
+// C ABI of the library (include/ssm.h): argument validation, variant choice,
+// TMA descriptor encoding and kernel launch. Nothing here allocates, frees or
+// synchronises (except ssm_device_error, which documents it).
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/ssm.h"
+#include "launch.h"
+#include "scan_params.h"
+
+namespace {
+
+thread_local std::string g_detail;
+
+ssm_status_t fail(ssm_status_t s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_detail = buf;
+    return s;
+}
+
+ssm_status_t ok() {
+    g_detail.clear();
+    return SSM_OK;
+}
+
+ssm_status_t cuda_fail(cudaError_t e, const char* what) {
+    return fail(SSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_size(ssm_dtype_t t) { return t == SSM_BF16 ? 2 : 4; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    auto x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// ------------------------------------------------------------ TMA encoding --
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D tile map over a row-major (d2, d1, d0) tensor, d0 innermost.
+bool encode_3d(CUtensorMap* map, int es, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    3, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- scan plan --
+
+struct ScanPlan {
+    ssm::ScanVariant v;
+    int mode;            // 0 fwd, 1 rev, 2 bidir
+    int nchunks;
+    int chunk_len;
+    size_t summary_bytes;
+    size_t partial_bytes;
+    size_t workspace;
+};
+
+int env_int(const char* name, int dflt) {
+    const char* s = std::getenv(name);
+    return s ? std::atoi(s) : dflt;
+}
+
+ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
+    if (!a) return fail(SSM_ERR_NULL_ARG, "args is NULL");
+    if (a->dtype != SSM_F32 && a->dtype != SSM_BF16)
+        return fail(SSM_ERR_BAD_DTYPE, "dtype %d is not SSM_F32 or SSM_BF16", (int)a->dtype);
+    if (a->batch < 0 || a->dim < 0 || a->seqlen < 0)
+        return fail(SSM_ERR_BAD_SHAPE, "negative size (batch %lld, dim %lld, seqlen %lld)",
+                    (long long)a->batch, (long long)a->dim, (long long)a->seqlen);
+    if (a->dstate < 1 || a->dstate > SSM_MAX_DSTATE)
+        return fail(SSM_ERR_BAD_SHAPE, "dstate %lld outside 1..%d", (long long)a->dstate,
+                    SSM_MAX_DSTATE);
+    if (a->seqlen > 0x3fffffffLL || a->dim > 0x3fffffffLL)
+        return fail(SSM_ERR_BAD_SHAPE, "seqlen and dim must be below 2^30");
+    if (a->batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch %lld > 65535", (long long)a->batch);
+    if (a->conv_weight && (a->conv_width < 1 || a->conv_width > SSM_MAX_CONV_WIDTH))
+        return fail(SSM_ERR_BAD_SHAPE, "conv_width %d outside 1..%d", a->conv_width,
+                    SSM_MAX_CONV_WIDTH);
+    if (a->num_chunks < 0) return fail(SSM_ERR_BAD_SHAPE, "num_chunks %d < 0", a->num_chunks);
+    const bool bidir = a->A_rev != nullptr;
+    if (a->final_state_rev && !bidir)
+        return fail(SSM_ERR_UNSUPPORTED, "final_state_rev needs A_rev (bidirectional)");
+    if (bidir && a->num_chunks > 1)
+        return fail(SSM_ERR_UNSUPPORTED, "the bidirectional sum runs as a single pass");
+
+    const int es = elem_size(a->dtype);
+    const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
+    int np = 4, s = 4;
+    if (ns == 16) {
+        // 8 lanes per channel doubles the warps when batch*dim alone leaves the SMs short
+        const int64_t warps4 = a->batch * a->dim * 4 / 32;
+        s = env_int("SSM_LANES_PER_CHANNEL", warps4 >= 2 * 4 * 148 ? 4 : 8);
+        if (s != 4 && s != 8) s = 4;
+        np = 16 / s;
+    } else if (ns == 8) {
+        np = 2;
+    } else {
+        np = 1;
+    }
+    if (!ssm::scan_variant(es, np, s, &pl->v))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for elem %d np %d s %d", es, np, s);
+    pl->mode = bidir ? 2 : (a->reverse ? 1 : 0);
+
+    const int tile = pl->v.tile;
+    const int64_t ntiles = (a->seqlen + tile - 1) / tile;
+    int nch = a->num_chunks;
+    if (nch == 0) nch = 1;
+    if (nch > ntiles) nch = (int)(ntiles > 0 ? ntiles : 1);
+    if (nch > 65535) nch = 65535;
+    const int64_t tiles_per_chunk = ntiles > 0 ? (ntiles + nch - 1) / nch : 1;
+    pl->chunk_len = (int)(tiles_per_chunk * tile);
+    pl->nchunks = ntiles > 0 ? (int)((ntiles + tiles_per_chunk - 1) / tiles_per_chunk) : 1;
+
+    const int64_t rows = a->batch * a->dim;
+    pl->summary_bytes =
+        pl->nchunks > 1 ? (size_t)(pl->nchunks - 1) * rows * ns * sizeof(float) * 2 : 0;
+    pl->partial_bytes = (bidir && a->dtype != SSM_F32) ? (size_t)rows * a->seqlen * 4 : 0;
+    // layout: [summaries][pad to 256][bidirectional fp32 partial]
+    pl->workspace = pl->partial_bytes ? ((pl->summary_bytes + 255) / 256) * 256 + pl->partial_bytes
+                                      : pl->summary_bytes;
+    return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_abi_version(void) { return SSM_ABI_VERSION; }
+
+const char* ssm_status_string(ssm_status_t s) {
+    switch (s) {
+        case SSM_OK: return "ok";
+        case SSM_ERR_NULL_ARG: return "a required pointer is NULL";
+        case SSM_ERR_BAD_SHAPE: return "a size is out of range";
+        case SSM_ERR_BAD_DTYPE: return "unknown dtype";
+        case SSM_ERR_MISALIGNED: return "a pointer is not aligned to its element size";
+        case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSM_ERR_UNSUPPORTED: return "unsupported combination of arguments";
+        case SSM_ERR_CUDA: return "CUDA runtime error";
+        case SSM_ERR_TIMEOUT: return "a kernel-side bounded wait ran out";
+        case SSM_ERR_ALIAS: return "output overlaps an input";
+    }
+    return "unknown status";
+}
+
+const char* ssm_last_error_detail(void) { return g_detail.c_str(); }
+
+ssm_status_t ssm_selective_scan_workspace_size(const ssm_scan_args_t* a, size_t* bytes) {
+    if (!bytes) return fail(SSM_ERR_NULL_ARG, "bytes is NULL");
+    ScanPlan pl;
+    ssm_status_t st = plan_scan(a, &pl);
+    if (st != SSM_OK) return st;
+    *bytes = pl.workspace;
+    return ok();
+}
+
+ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t stream) {
+    ScanPlan pl;
+    ssm_status_t st = plan_scan(a, &pl);
+    if (st != SSM_OK) return st;
+    const bool bidir = pl.mode == 2;
+    const int es = elem_size(a->dtype);
+    const int64_t rows = a->batch * a->dim;
+    const size_t act = (size_t)rows * a->seqlen * es;
+    const size_t bc = (size_t)a->batch * a->dstate * a->seqlen * es;
+    const bool empty = rows == 0 || a->seqlen == 0;
+
+    if (!empty) {
+        struct { const void* p; const char* n; } req[] = {
+            {a->u, "u"}, {a->delta, "delta"}, {a->A, "A"}, {a->B, "B"}, {a->C, "C"},
+            {a->out, "out"}};
+        for (auto& r : req)
+            if (!r.p) return fail(SSM_ERR_NULL_ARG, "%s is NULL", r.n);
+    }
+    // element alignment
+    struct { const void* p; size_t al; const char* n; } al[] = {
+        {a->u, (size_t)es, "u"}, {a->delta, (size_t)es, "delta"}, {a->z, (size_t)es, "z"},
+        {a->B, (size_t)es, "B"}, {a->C, (size_t)es, "C"}, {a->out, (size_t)es, "out"},
+        {a->A, 4, "A"}, {a->D, 4, "D"}, {a->delta_bias, 4, "delta_bias"},
+        {a->conv_weight, 4, "conv_weight"}, {a->conv_bias, 4, "conv_bias"},
+        {a->A_rev, 4, "A_rev"}, {a->D_rev, 4, "D_rev"}, {a->delta_bias_rev, 4, "delta_bias_rev"},
+        {a->final_state, 4, "final_state"}, {a->final_state_rev, 4, "final_state_rev"},
+        {a->workspace, 16, "workspace"}};
+    for (auto& x : al)
+        if (x.p && !aligned(x.p, x.al))
+            return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", x.n, x.al);
+    if (!empty) {
+        if (overlap(a->out, act, a->u, act) || overlap(a->out, act, a->delta, act) ||
+            overlap(a->out, act, a->z, act) || overlap(a->out, act, a->B, bc) ||
+            overlap(a->out, act, a->C, bc))
+            return fail(SSM_ERR_ALIAS, "out overlaps an input");
+    }
+    if (pl.workspace > 0 && (!a->workspace || a->workspace_bytes < pl.workspace))
+        return fail(SSM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.workspace,
+                    a->workspace ? a->workspace_bytes : (size_t)0);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (empty) {
+        // zero steps: the final state is the (zero) initial state
+        const size_t fs = (size_t)rows * a->dstate * sizeof(float);
+        if (fs && a->final_state) {
+            cudaError_t e = cudaMemsetAsync(a->final_state, 0, fs, s);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+        }
+        if (fs && a->final_state_rev) {
+            cudaError_t e = cudaMemsetAsync(a->final_state_rev, 0, fs, s);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+        }
+        return ok();
+    }
+
+    ssm::ScanParams p{};
+    p.batch = (int)a->batch;
+    p.dim = (int)a->dim;
+    p.seqlen = (int)a->seqlen;
+    p.dstate = (int)a->dstate;
+    p.u = a->u;
+    p.delta = a->delta;
+    p.z = a->z;
+    p.Bm = a->B;
+    p.Cm = a->C;
+    p.A[0] = a->A;
+    p.Dv[0] = a->D;
+    p.dbias[0] = a->delta_bias;
+    p.A[1] = bidir ? a->A_rev : a->A;
+    p.Dv[1] = bidir ? a->D_rev : a->D;
+    p.dbias[1] = bidir ? a->delta_bias_rev : a->delta_bias;
+    p.conv_w = a->conv_weight;
+    p.conv_b = a->conv_weight ? a->conv_bias : nullptr;
+    p.conv_width = a->conv_weight ? a->conv_width : 0;
+    p.softplus = a->delta_softplus ? 1 : 0;
+    p.mode = pl.mode;
+    p.out = a->out;
+    p.final_state[0] = a->final_state;
+    p.final_state[1] = a->final_state_rev;
+    p.chunk_len = pl.chunk_len;
+    p.nchunks = pl.nchunks;
+    uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+    p.summary = pl.summary_bytes ? reinterpret_cast<float2*>(ws) : nullptr;
+    if (bidir)
+        p.partial = a->dtype == SSM_F32
+                        ? static_cast<float*>(a->out)
+                        : reinterpret_cast<float*>(ws + ((pl.summary_bytes + 255) / 256) * 256);
+    const bool row16 = (a->seqlen * es) % 16 == 0;
+    p.vec_store = row16 && aligned(a->out, 16);
+
+    // TMA needs 16-byte row strides and 16-byte aligned bases
+    bool tma = row16 && aligned(a->u, 16) && aligned(a->delta, 16) && aligned(a->B, 16) &&
+               aligned(a->C, 16) && (!a->z || aligned(a->z, 16)) && env_int("SSM_NO_TMA", 0) == 0;
+    ssm::ScanMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (tma) {
+        const auto& v = pl.v;
+        const uint32_t xbox = a->conv_weight ? v.tile + v.halo : v.tile;
+        const uint64_t L = a->seqlen, D = a->dim, Bn = a->batch, N = a->dstate;
+        // B, C tiles use the swizzle whose span equals one tile row (64 B bf16, 128 B fp32)
+        const CUtensorMapSwizzle bc =
+            v.tile * es == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+        const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+        tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
+              encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
+              (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, none)) &&
+              encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
+              encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc);
+    }
+
+    const unsigned gx = (unsigned)((a->dim + pl.v.channels - 1) / pl.v.channels);
+    cudaError_t e;
+    if (pl.nchunks > 1) {
+        e = ssm::launch_scan(pl.v, tma, true, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
+                             s);
+        if (e != cudaSuccess) return cuda_fail(e, "summary pass launch");
+    }
+    e = ssm::launch_scan(pl.v, tma, false, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return ok();
+}
+
+ssm_status_t ssm_causal_conv1d_fwd(const void* x, const float* w, const float* bias, void* out,
+                                   int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
+                                   int32_t apply_silu, ssm_dtype_t dtype, ssm_stream_t stream) {
+    if (dtype != SSM_F32 && dtype != SSM_BF16)
+        return fail(SSM_ERR_BAD_DTYPE, "dtype %d is not SSM_F32 or SSM_BF16", (int)dtype);
+    if (batch < 0 || dim < 0 || seqlen < 0)
+        return fail(SSM_ERR_BAD_SHAPE, "negative size");
+    if (width < 1 || width > SSM_MAX_CONV_WIDTH)
+        return fail(SSM_ERR_BAD_SHAPE, "width %d outside 1..%d", width, SSM_MAX_CONV_WIDTH);
+    if (seqlen > 0x3fffffffLL || dim > 0x3fffffffLL)
+        return fail(SSM_ERR_BAD_SHAPE, "seqlen and dim must be below 2^30");
+    const int64_t rows = batch * dim;
+    if (rows == 0 || seqlen == 0) return ok();
+    if (!x || !w || !out) return fail(SSM_ERR_NULL_ARG, "%s is NULL", !x ? "x" : !w ? "w" : "out");
+    const int es = elem_size(dtype);
+    if (!aligned(x, es) || !aligned(out, es) || !aligned(w, 4) || (bias && !aligned(bias, 4)))
+        return fail(SSM_ERR_MISALIGNED, "a pointer is not aligned to its element size");
+    const size_t n = (size_t)rows * seqlen * es;
+    if (overlap(x, n, out, n)) return fail(SSM_ERR_ALIAS, "out overlaps x");
+    ssm::ConvParams p{x, w, bias, out, rows, (int)dim, (int)seqlen, width, apply_silu ? 1 : 0};
+    const bool vec = (seqlen % 8 == 0) && aligned(x, 16) && aligned(out, 16);
+    cudaError_t e = ssm::launch_conv(es, vec, p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "conv launch");
+    return ok();
+}
+
+ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const void* x,
+                                        const void* dt, const float* A, const void* B_t,
+                                        const void* C_t, const float* D, const void* z,
+                                        const float* dt_bias, int32_t dt_softplus,
+                                        const float* conv_weight, const float* conv_bias,
+                                        int32_t conv_width, void* out, int64_t batch,
+                                        int64_t dim, int64_t dstate, ssm_dtype_t dtype,
+                                        ssm_stream_t stream) {
+    if (dtype != SSM_F32 && dtype != SSM_BF16)
+        return fail(SSM_ERR_BAD_DTYPE, "dtype %d is not SSM_F32 or SSM_BF16", (int)dtype);
+    if (batch < 0 || dim < 0) return fail(SSM_ERR_BAD_SHAPE, "negative size");
+    if (dstate < 1 || dstate > SSM_MAX_DSTATE)
+        return fail(SSM_ERR_BAD_SHAPE, "dstate %lld outside 1..%d", (long long)dstate,
+                    SSM_MAX_DSTATE);
+    if (conv_weight && (conv_width < 1 || conv_width > SSM_MAX_CONV_WIDTH))
+        return fail(SSM_ERR_BAD_SHAPE, "conv_width %d outside 1..%d", conv_width,
+                    SSM_MAX_CONV_WIDTH);
+    if (dim > 0x3fffffffLL) return fail(SSM_ERR_BAD_SHAPE, "dim must be below 2^30");
+    const int64_t rows = batch * dim;
+    if (rows == 0) return ok();
+    struct { const void* p; const char* n; } req[] = {
+        {state, "state"}, {x, "x"}, {dt, "dt"}, {A, "A"}, {B_t, "B_t"}, {C_t, "C_t"}, {out, "out"}};
+    for (auto& r : req)
+        if (!r.p) return fail(SSM_ERR_NULL_ARG, "%s is NULL", r.n);
+    if (conv_weight && !conv_state) return fail(SSM_ERR_NULL_ARG, "conv_state is NULL");
+    const int es = elem_size(dtype);
+    struct { const void* p; size_t al; const char* n; } al[] = {
+        {state, 4, "state"}, {conv_state, (size_t)es, "conv_state"}, {x, (size_t)es, "x"},
+        {dt, (size_t)es, "dt"}, {A, 4, "A"}, {B_t, (size_t)es, "B_t"}, {C_t, (size_t)es, "C_t"},
+        {D, 4, "D"}, {z, (size_t)es, "z"}, {dt_bias, 4, "dt_bias"},
+        {conv_weight, 4, "conv_weight"}, {conv_bias, 4, "conv_bias"}, {out, (size_t)es, "out"}};
+    for (auto& q : al)
+        if (q.p && !aligned(q.p, q.al))
+            return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", q.n, q.al);
+    const size_t on = (size_t)rows * es;
+    if (overlap(out, on, x, on) || overlap(out, on, dt, on) || overlap(out, on, z, on) ||
+        overlap(out, on, state, (size_t)rows * dstate * 4))
+        return fail(SSM_ERR_ALIAS, "out overlaps an input");
+    ssm::DecodeParams p{};
+    p.state = state;
+    p.conv_state = conv_weight ? conv_state : nullptr;
+    p.x = x;
+    p.dt = dt;
+    p.A = A;
+    p.Bt = B_t;
+    p.Ct = C_t;
+    p.D = D;
+    p.z = z;
+    p.dt_bias = dt_bias;
+    p.conv_w = conv_weight;
+    p.conv_b = conv_weight ? conv_bias : nullptr;
+    p.out = out;
+    p.rows = rows;
+    p.dim = (int)dim;
+    p.dstate = (int)dstate;
+    p.conv_width = conv_weight ? conv_width : 0;
+    p.softplus = dt_softplus ? 1 : 0;
+    p.vec = dstate == 16 && aligned(state, 16) && aligned(A, 16);
+    cudaError_t e = ssm::launch_decode(es, (int)dstate, p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+    return ok();
+}
+
+ssm_status_t ssm_device_error(int32_t* code, ssm_stream_t stream) {
+    if (!code) return fail(SSM_ERR_NULL_ARG, "code is NULL");
+    int c = 0;
+    cudaError_t e = ssm::read_device_error(&c, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    *code = c;
+    return ok();
+}
+
+}  // extern "C"
