@@ -9,7 +9,7 @@ import torch
 import oracle
 import mamba_selective_scan_sm_b200 as ssm
 from mamba_selective_scan_sm_b200 import synth
-from tests.gpu_helpers import assert_close, dev, host, state_close
+from tests.gpu_helpers import assert_close_out, dev, host, state_close
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -41,7 +41,7 @@ def _check(w, res, inp, chans):
     y = res[0]
     rows = torch.tensor([b * w.dim + d for b, d in chans], device="cuda")
     yg = host(y.reshape(-1, w.seqlen)[rows])
-    assert_close(yg, ref[0], w.dtype, w.name)
+    assert_close_out(yg, ref[0], w.dtype, w.name)
     hg = host(res[1].reshape(-1, res[1].shape[-1])[rows])
     state_close(hg, ref[1], "final state")
     if w.bidirectional:
@@ -96,5 +96,5 @@ def test_fullsize_decode_64_steps():
                 inp["C"][s, b:b + 1], inp["D"][d:d + 1], sl("z"), inp["dt_bias"][d:d + 1], True,
                 inp["conv_w"][d:d + 1], inp["conv_b"][d:d + 1])
             yo.append(y[0, 0])
-        assert_close(og[:, b, d], np.array(yo), "bf16", f"decode channel {(b, d)}")
+        assert_close_out(og[:, b, d], np.array(yo), "bf16", f"decode channel {(b, d)}")
         state_close(sg[b, d], so[0, 0], "state")
