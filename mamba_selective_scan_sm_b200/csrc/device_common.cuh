@@ -48,6 +48,34 @@ __device__ __forceinline__ float softplus(float x) {
 // silu(v) = v * sigmoid(v) = v / (1 + e^-v); tends to 0 for v -> -inf.
 __device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
 
+// ------------------------------------------------------ packed fp32 pairs --
+// sm_100 executes add/mul/fma on two fp32 lanes of a 64-bit register pair as one
+// instruction (.f32x2); the pipe throughput per element is unchanged, but issue
+// slots are halved.
+
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 upk2(uint64_t r) {
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ float lo2(uint64_t r) { return upk2(r).x; }
+__device__ __forceinline__ float hi2(uint64_t r) { return upk2(r).y; }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // ------------------------------------------------------- shared / barriers --
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -24,6 +24,8 @@
 // launch starts chunk k from the carry H_k = P_{k-1} H_{k-1} + S_{k-1}.
 #pragma once
 
+#include <type_traits>
+
 #include "device_common.cuh"
 #include "scan_params.h"
 
@@ -77,8 +79,73 @@ __device__ __forceinline__ int swz(int row, int byte_in_row) {
     return off ^ (((off >> 7) & SWZ) << 4);
 }
 
+// Recurrence state of one lane: NP states, held as fp32 pairs so the four
+// per-state operations (delta*A, delta*u*B, the h update and C.h) issue as packed
+// .f32x2 instructions.
+template <int NP, bool SUMMARY>
+struct LaneState {
+    static constexpr int NPR = NP / 2;                   // packed pairs
+    static constexpr bool ODD = (NP % 2) != 0;
+    uint64_t h2[NPR > 0 ? NPR : 1], a2[NPR > 0 ? NPR : 1], pr2[NPR > 0 ? NPR : 1];
+    float h1, a1, pr1;                                   // the unpaired state (NP odd)
+
+    __device__ __forceinline__ void set_a(const float* a) {
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) a2[k] = pk2(a[2 * k], a[2 * k + 1]);
+        if (ODD) a1 = a[NP - 1];
+    }
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) { h2[k] = pk2(0.f, 0.f); pr2[k] = pk2(1.f, 1.f); }
+        h1 = 0.f;
+        pr1 = 1.f;
+    }
+    __device__ __forceinline__ float get(int k) const {       // k is a compile-time index
+        if (ODD && k == NP - 1) return h1;
+        return (k & 1) ? hi2(h2[k >> 1]) : lo2(h2[k >> 1]);
+    }
+    __device__ __forceinline__ float get_pr(int k) const {
+        if (ODD && k == NP - 1) return pr1;
+        return (k & 1) ? hi2(pr2[k >> 1]) : lo2(pr2[k >> 1]);
+    }
+    __device__ __forceinline__ void set(const float* v) {
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) h2[k] = pk2(v[2 * k], v[2 * k + 1]);
+        if (ODD) h1 = v[NP - 1];
+    }
+
+    // One time step: h = exp2(delta*a2) * h + (delta*u) * B; returns sum_k C_k h_k.
+    // bv / cv point at this lane's NP consecutive fp32 B and C values of the step.
+    __device__ __forceinline__ float step(float dl, float du, const float* bv, const float* cv) {
+        const uint64_t dd = pk2(dl, dl), uu = pk2(du, du);
+        uint64_t s = pk2(0.f, 0.f);
+        float s1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) {
+            const float2 bb = *reinterpret_cast<const float2*>(bv + 2 * k);
+            const uint64_t x = mul2(dd, a2[k]);
+            const uint64_t dA = pk2(ex2(lo2(x)), ex2(hi2(x)));
+            h2[k] = fma2(dA, h2[k], mul2(uu, pk2(bb.x, bb.y)));
+            if (SUMMARY) {
+                pr2[k] = mul2(pr2[k], dA);
+            } else {
+                const float2 cc = *reinterpret_cast<const float2*>(cv + 2 * k);
+                s = fma2(pk2(cc.x, cc.y), h2[k], s);
+            }
+        }
+        if (ODD) {
+            const float dA = ex2(dl * a1);
+            h1 = fmaf(dA, h1, du * bv[NP - 1]);
+            if (SUMMARY) pr1 *= dA;
+            else s1 = cv[NP - 1] * h1;
+        }
+        return (NPR > 0 ? lo2(s) + hi2(s) : 0.f) + s1;
+    }
+};
+
+// At most 128 registers per thread, so four 128-thread CTAs fit an SM's register file.
 template <typename T, int NP, int S, bool USE_TMA, bool SUMMARY>
-__global__ void __launch_bounds__(kScanThreads)
+__global__ void __launch_bounds__(kScanThreads, 4)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     using Cfg = ScanCfg<T, NP, S>;
     using E = Elem<T>;
@@ -202,40 +269,51 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    float h[NP], a2[NP], pr[NP];
+    LaneState<NP, SUMMARY> ls;
     auto load_A = [&](int dir) {
+        float a[NP];
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
             const int n = j * NP + k;
-            a2[k] = (dvalid && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
+            a[k] = (dvalid && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
         }
+        ls.set_a(a);
     };
     // Initial state of this chunk: carry over the summaries of earlier chunks.
     auto init_state = [&]() {
-#pragma unroll
-        for (int k = 0; k < NP; ++k) { h[k] = 0.f; pr[k] = 1.f; }
+        ls.reset();
         if (!SUMMARY && chunk > 0 && dvalid) {
+            float hv[NP];
+#pragma unroll
+            for (int k = 0; k < NP; ++k) hv[k] = 0.f;
             const int64_t stride = (int64_t)p.batch * p.dim * NS;
             for (int k2 = 0; k2 < chunk; ++k2) {
                 const float2* sm = p.summary + k2 * stride + row * NS + j * NP;
 #pragma unroll
                 for (int k = 0; k < NP; ++k) {
                     const float2 ps = sm[k];
-                    h[k] = fmaf(ps.x, h[k], ps.y);
+                    hv[k] = fmaf(ps.x, hv[k], ps.y);
                 }
             }
+            ls.set(hv);
         }
     };
 
     auto prologue = [&](int f, const uint8_t* st) {
         const bool rv = tile_rev(f);
         const int xoff = (conv && !rv) ? HALO : 0;
-        // B, C: swizzled [n][t] (input dtype) -> [t][n] fp32
-        for (int e = tid; e < NS * TT; e += kScanThreads) {
-            const int n = e % NS, tt = e / NS;
-            const int off = swz<ROWB, SWZ>(n, tt * (int)sizeof(T));
-            Bt[tt * NS + n] = E::to_f(*reinterpret_cast<const T*>(st + Cfg::RAW_B + off));
-            Ct[tt * NS + n] = E::to_f(*reinterpret_cast<const T*>(st + Cfg::RAW_C + off));
+        // B, C: swizzled [n][t] (input dtype) -> [t][n] fp32, one 16-byte chunk per thread
+        constexpr int EPC = 16 / (int)sizeof(T);           // elements per 16-byte chunk
+        constexpr int NCH = NS * ROWB / 16;                // chunks per tensor
+        for (int e = tid; e < 2 * NCH; e += kScanThreads) {
+            const int ten = e / NCH, ch = e % NCH;
+            const int n = ch % NS, t0 = (ch / NS) * EPC;
+            const uint8_t* src = st + (ten ? Cfg::RAW_C : Cfg::RAW_B) + swz<ROWB, SWZ>(n, t0 * (int)sizeof(T));
+            float* dst = (ten ? Ct : Bt) + t0 * NS + n;
+            const uint4 v = *reinterpret_cast<const uint4*>(src);
+            const T* tv = reinterpret_cast<const T*>(&v);
+#pragma unroll
+            for (int m = 0; m < EPC; ++m) dst[m * NS] = E::to_f(tv[m]);
         }
         // per (channel, t) quantities; a warp walks one channel row, lanes along t
         for (int idx = warp; idx < G * (TT / 32); idx += kScanThreads / 32) {
@@ -275,142 +353,119 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                                                           c * Cfg::P_PITCH);
     const float2* Erow = reinterpret_cast<const float2*>(reinterpret_cast<uint8_t*>(Ebuf) +
                                                           c * Cfg::E_PITCH);
+    const float* Bl = Bt + j * NP;
+    const float* Cl = Ct + j * NP;
 
-    auto scan_tile = [&](int f) {
-        const bool rv = tile_rev(f);
+    // gate, skip term, bidirectional partial and the store of R owned outputs
+    auto epilogue = [&](const float* acc, bool rv, int dir, int l0, int pos0, int nown) {
+        float yv[R];
+#pragma unroll
+        for (int m = 0; m < R; ++m) {
+            const int ii = pos0 + m;
+            const int tt = rv ? TT - 1 - ii : ii;
+            const float2 e = Erow[tt];
+            yv[m] = (acc[m] + e.x) * e.y;
+        }
+        if (!dvalid || nown <= 0) return;
+        const int tmin = rv ? l0 + TT - 1 - (pos0 + R - 1) : l0 + pos0;
+        float ya[R];                                      // time-ascending order
+#pragma unroll
+        for (int m = 0; m < R; ++m) ya[m] = rv ? yv[R - 1 - m] : yv[m];
+        // valid ascending index range: forward [0, nown); reverse [R - nown, R)
+        const int mlo = rv ? R - nown : 0;
+        const int mhi = rv ? R : nown;
+        const int64_t gbase = row * L + tmin;
+        if (p.mode == 2 && dir == 1) {
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+                if (m >= mlo && m < mhi) ya[m] += p.partial[gbase + m];
+        }
+        if (p.mode == 2 && dir == 0) {
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+                if (m >= mlo && m < mhi) p.partial[gbase + m] = ya[m];
+            return;
+        }
+        T* out = static_cast<T*>(p.out) + gbase;
+        const bool full = (mlo == 0 && mhi == R) && p.vec_store;
+        if (full && R * sizeof(T) == 16) {
+            if constexpr (sizeof(T) == 4) {
+                *reinterpret_cast<float4*>(out) = make_float4(ya[0], ya[1 % R], ya[2 % R], ya[3 % R]);
+            } else {
+                uint4 v;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    __nv_bfloat162 t2 = __floats2bfloat162_rn(ya[(2 * m) % R], ya[(2 * m + 1) % R]);
+                    w[m] = *reinterpret_cast<uint32_t*>(&t2);
+                }
+                *reinterpret_cast<uint4*>(out) = v;
+            }
+        } else if (full && R * sizeof(T) == 8) {
+            if constexpr (sizeof(T) == 4) {
+                *reinterpret_cast<float2*>(out) = make_float2(ya[0], ya[1 % R]);
+            } else {
+                __nv_bfloat162 t0 = __floats2bfloat162_rn(ya[0], ya[1 % R]);
+                __nv_bfloat162 t1 = __floats2bfloat162_rn(ya[2 % R], ya[3 % R]);
+                uint2 v;
+                v.x = *reinterpret_cast<uint32_t*>(&t0);
+                v.y = *reinterpret_cast<uint32_t*>(&t1);
+                *reinterpret_cast<uint2*>(out) = v;
+            }
+        } else if (full && R * sizeof(T) == 4 && sizeof(T) == 2) {
+            *reinterpret_cast<__nv_bfloat162*>(out) = __floats2bfloat162_rn(ya[0], ya[1 % R]);
+        } else {
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+                if (m >= mlo && m < mhi) out[m] = E::from_f(ya[m]);
+        }
+    };
+
+    // butterfly transpose-reduce over the S lanes of a channel: afterwards lane j
+    // holds the sums of block positions [j*R, j*R + R) in acc[0 .. R)
+    auto reduce_block = [&](float* acc) {
+        int len = 16;
+#pragma unroll
+        for (int m = S / 2; m >= 1; m >>= 1) {
+            const int half = len >> 1;
+            const bool upper = (j & m) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float send = upper ? acc[i] : acc[i + half];
+                const float keep = upper ? acc[i + half] : acc[i];
+                acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+            len = half;
+        }
+    };
+
+    // One tile in scan order. RV: walk time downwards. FULL: all TT steps valid
+    // (no per-step predicate; shared-memory offsets are compile-time constants).
+    auto scan_tile = [&](auto rv_tag, auto full_tag, int f) {
+        constexpr bool RV = decltype(rv_tag)::value;
+        constexpr bool FULL = decltype(full_tag)::value;
         const int dir = (p.mode == 2 && f >= ntl) ? 1 : 0;
-        const int jt = f % ntl;
-        const int i0 = cs + jt * TT;
-        const int nvalid = min(TT, ce - i0);
-        const int l0 = rv ? L - i0 - TT : i0;
+        const int i0 = cs + (f % ntl) * TT;
+        const int nvalid = FULL ? TT : min(TT, ce - i0);
+        const int l0 = RV ? L - i0 - TT : i0;
 #pragma unroll 1
         for (int blk = 0; blk < TT / 16; ++blk) {
-            if (blk * 16 >= nvalid) break;
+            if (!FULL && blk * 16 >= nvalid) break;
             float acc[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
                 const int ii = blk * 16 + q;
-                const int tt = rv ? TT - 1 - ii : ii;
+                const int tt = RV ? TT - 1 - ii : ii;
                 acc[q] = 0.f;
-                if (ii < nvalid) {
+                if (FULL || ii < nvalid) {
                     const float2 pd = Prow[tt];
-                    float bv[NP], cv[NP];
-                    if constexpr (NP == 4) {
-                        const float4 b4 = *reinterpret_cast<const float4*>(Bt + tt * NS + j * 4);
-                        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
-                        if (!SUMMARY) {
-                            const float4 c4 = *reinterpret_cast<const float4*>(Ct + tt * NS + j * 4);
-                            cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
-                        }
-                    } else if constexpr (NP == 2) {
-                        const float2 b2 = *reinterpret_cast<const float2*>(Bt + tt * NS + j * 2);
-                        bv[0] = b2.x; bv[1] = b2.y;
-                        if (!SUMMARY) {
-                            const float2 c2 = *reinterpret_cast<const float2*>(Ct + tt * NS + j * 2);
-                            cv[0] = c2.x; cv[1] = c2.y;
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < NP; ++k) {
-                            bv[k] = Bt[tt * NS + j * NP + k];
-                            if (!SUMMARY) cv[k] = Ct[tt * NS + j * NP + k];
-                        }
-                    }
-                    float a = 0.f;
-#pragma unroll
-                    for (int k = 0; k < NP; ++k) {
-                        const float dA = ex2(pd.x * a2[k]);
-                        h[k] = fmaf(dA, h[k], pd.y * bv[k]);
-                        if (SUMMARY) pr[k] *= dA;
-                        else a = fmaf(cv[k], h[k], a);
-                    }
-                    acc[q] = a;
+                    acc[q] = ls.step(pd.x, pd.y, Bl + tt * NS, Cl + tt * NS);
                 }
             }
             if (SUMMARY) continue;
-            // butterfly transpose-reduce over the S lanes of the channel:
-            // afterwards lane j holds the sums for block positions [j*R, j*R + R)
-            int len = 16;
-#pragma unroll
-            for (int m = S / 2; m >= 1; m >>= 1) {
-                const int half = len >> 1;
-                const bool upper = (j & m) != 0;
-#pragma unroll
-                for (int i = 0; i < half; ++i) {
-                    const float send = upper ? acc[i] : acc[i + half];
-                    const float keep = upper ? acc[i + half] : acc[i];
-                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
-                len = half;
-            }
-            // epilogue: gate, skip term, (bidirectional partial), store R outputs
-            const int pos0 = blk * 16 + j * R;             // first owned position in tile
-            float yv[R];
-            int tmin;                                      // smallest time among them
-#pragma unroll
-            for (int m = 0; m < R; ++m) {
-                const int ii = pos0 + m;
-                const int tt = rv ? TT - 1 - ii : ii;
-                const float2 e = Erow[tt];
-                yv[m] = (acc[m] + e.x) * e.y;
-            }
-            tmin = rv ? l0 + TT - 1 - (pos0 + R - 1) : l0 + pos0;
-            const int nown = max(0, min(R, nvalid - pos0));
-            if (dvalid && nown > 0) {
-                // time-ascending order
-                float ya[R];
-#pragma unroll
-                for (int m = 0; m < R; ++m) ya[m] = rv ? yv[R - 1 - m] : yv[m];
-                // valid ascending index range: forward [0, nown); reverse [R - nown, R)
-                const int mlo = rv ? R - nown : 0;
-                const int mhi = rv ? R : nown;
-                const int64_t gbase = row * L + tmin;
-                if (p.mode == 2 && dir == 1) {
-#pragma unroll
-                    for (int m = 0; m < R; ++m)
-                        if (m >= mlo && m < mhi) ya[m] += p.partial[gbase + m];
-                }
-                if (p.mode == 2 && dir == 0) {
-#pragma unroll
-                    for (int m = 0; m < R; ++m)
-                        if (m >= mlo && m < mhi) p.partial[gbase + m] = ya[m];
-                } else {
-                    T* out = static_cast<T*>(p.out) + gbase;
-                    const bool full = (mlo == 0 && mhi == R) && p.vec_store;
-                    if (full && R * sizeof(T) == 16) {
-                        if constexpr (sizeof(T) == 4) {
-                            *reinterpret_cast<float4*>(out) = make_float4(ya[0], ya[1 % R], ya[2 % R], ya[3 % R]);
-                        } else {
-                            uint4 v;
-                            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) {
-                                __nv_bfloat162 t2 = __floats2bfloat162_rn(ya[(2 * m) % R], ya[(2 * m + 1) % R]);
-                                w[m] = *reinterpret_cast<uint32_t*>(&t2);
-                            }
-                            *reinterpret_cast<uint4*>(out) = v;
-                        }
-                    } else if (full && R * sizeof(T) == 8) {
-                        if constexpr (sizeof(T) == 4) {
-                            *reinterpret_cast<float2*>(out) = make_float2(ya[0], ya[1 % R]);
-                        } else {
-                            __nv_bfloat162 t0 = __floats2bfloat162_rn(ya[0], ya[1 % R]);
-                            __nv_bfloat162 t1 = __floats2bfloat162_rn(ya[2 % R], ya[3 % R]);
-                            uint2 v;
-                            v.x = *reinterpret_cast<uint32_t*>(&t0);
-                            v.y = *reinterpret_cast<uint32_t*>(&t1);
-                            *reinterpret_cast<uint2*>(out) = v;
-                        }
-                    } else if (full && R * sizeof(T) == 4 && sizeof(T) == 2) {
-                        *reinterpret_cast<__nv_bfloat162*>(out) =
-                            __floats2bfloat162_rn(ya[0], ya[1 % R]);
-                    } else {
-#pragma unroll
-                        for (int m = 0; m < R; ++m)
-                            if (m >= mlo && m < mhi) out[m] = E::from_f(ya[m]);
-                    }
-                }
-            }
+            reduce_block(acc);
+            const int pos0 = blk * 16 + j * R;
+            epilogue(acc, RV, dir, l0, pos0, FULL ? R : max(0, min(R, nvalid - pos0)));
         }
     };
 
@@ -419,13 +474,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         if (SUMMARY) {
             float2* sm = p.summary + (int64_t)chunk * p.batch * p.dim * NS + row * NS + j * NP;
 #pragma unroll
-            for (int k = 0; k < NP; ++k) sm[k] = make_float2(pr[k], h[k]);
+            for (int k = 0; k < NP; ++k) sm[k] = make_float2(ls.get_pr(k), ls.get(k));
         } else if (chunk == p.nchunks - 1 && p.final_state[dir]) {
             float* fs = p.final_state[dir] + row * p.dstate;
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const int n = j * NP + k;
-                if (n < p.dstate) fs[n] = h[k];
+                if (n < p.dstate) fs[n] = ls.get(k);
             }
         }
     };
@@ -447,8 +502,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             __syncthreads();                 // params of direction 0 no longer read
             load_params(1);
             load_A(1);
-#pragma unroll
-            for (int k = 0; k < NP; ++k) { h[k] = 0.f; pr[k] = 1.f; }
+            ls.reset();
             __syncthreads();
         }
         bool ok = true;
@@ -470,7 +524,17 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             return;
         }
         if (USE_TMA && tid == 0 && f + NSTAGE < nt) issue(f + NSTAGE);
-        scan_tile(f);
+        const bool rv = tile_rev(f);
+        const bool full = cs + (f % ntl) * TT + TT <= ce;
+        using TrueT = std::integral_constant<bool, true>;
+        using FalseT = std::integral_constant<bool, false>;
+        if (full) {
+            if (rv) scan_tile(TrueT{}, TrueT{}, f);
+            else scan_tile(FalseT{}, TrueT{}, f);
+        } else {
+            if (rv) scan_tile(TrueT{}, FalseT{}, f);
+            else scan_tile(FalseT{}, FalseT{}, f);
+        }
         __syncthreads();
     }
     finish_direction(p.mode == 2 ? 1 : 0);
