@@ -172,6 +172,30 @@ SSM_API ssm_status_t ssm_selective_state_update(float* state, void* conv_state, 
                                         int64_t dim, int64_t dstate, ssm_dtype_t dtype,
                                         ssm_stream_t stream);
 
+/*
+ * Selective-scan forward that allocates nothing (the pages have no counterpart:
+ * this is a deployment convenience). Same arguments and results as
+ * ssm_selective_scan_fwd, except that `workspace` / `workspace_bytes` are ignored:
+ * the scratch the call needs (two-pass chunk summaries, the bf16 bidirectional
+ * partial) lives in a fixed device array of SSM_NOALLOC_SCRATCH_BYTES compiled
+ * into the library, which every GPU that loads the library holds until exit.
+ * For callers that cannot call cudaMalloc (a runtime that hands out only fixed
+ * buffers, a C caller with no allocator, a loop that must not risk an allocation's
+ * implicit synchronisation).
+ *  - A call needing more scratch than SSM_NOALLOC_SCRATCH_BYTES returns
+ *    SSM_ERR_WORKSPACE and launches nothing.
+ *  - The first call on each device looks the array's address up
+ *    (cudaGetSymbolAddress, with that device current); make that first call before
+ *    any stream capture. It allocates nothing, and neither do later calls.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents; nothing in it needs to start at zero (each launch writes its
+ *    scratch before reading it). Calls whose kernels overlap on the GPU (other
+ *    streams, other threads) race on it: serialise them.
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (8u << 20)
+SSM_API ssm_status_t ssm_selective_scan_fwd_noalloc(const ssm_scan_args_t* args,
+                                                    ssm_stream_t stream);
+
 /* Read and clear the device-side error word (0 = none; 1 = a bounded wait ran out).
  * Synchronises `stream`. */
 SSM_API ssm_status_t ssm_device_error(int32_t* code, ssm_stream_t stream);

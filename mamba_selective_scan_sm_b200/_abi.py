@@ -19,8 +19,9 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTS = (
     "ssm_abi_version", "ssm_status_string", "ssm_last_error_detail", "ssm_causal_conv1d_fwd",
     "ssm_selective_scan_workspace_size", "ssm_selective_scan_fwd", "ssm_selective_state_update",
-    "ssm_device_error",
+    "ssm_device_error", "ssm_selective_scan_fwd_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _P = ctypes.c_void_p
 _FP = ctypes.POINTER(ctypes.c_float)
@@ -77,6 +78,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_selective_state_update.restype = ctypes.c_int
     lib.ssm_selective_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P,
                                                _P, _I32, _P, _I64, _I64, _I64, ctypes.c_int, _P]
+    lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssm_selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _P]
     lib.ssm_device_error.restype = ctypes.c_int
     lib.ssm_device_error.argtypes = [ctypes.POINTER(_I32), _P]
     if path == LIB_PATH:

@@ -28,6 +28,9 @@ cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream
 
 cudaError_t launch_decode(int elem_size, int dstate, const DecodeParams& p, cudaStream_t stream);
 
+// Replace the calling thread's ssm_last_error_detail() text.
+void set_error_detail(const char* text);
+
 // Read and clear the device error word (synchronises `stream`).
 cudaError_t read_device_error(int* code, cudaStream_t stream);
 

@@ -161,6 +161,8 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
 
 }  // namespace
 
+void ssm::set_error_detail(const char* text) { g_detail = text ? text : ""; }
+
 extern "C" {
 
 int ssm_abi_version(void) { return SSM_ABI_VERSION; }
