@@ -91,6 +91,37 @@ def exp_count(w) -> int:
     return w.batch * w.dim * steps * w.dstate * dirs
 
 
+# ---------------------------------------------------------------- traffic --
+
+def kernel_source_digest() -> str:
+    """sha256 over the CUDA sources of the library (what an ncu capture describes)."""
+    import hashlib
+    d = os.path.join(ROOT, "mamba_selective_scan_sm_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(w):
+    """DRAM bytes (read + write) per launch of the workload's dominant kernel, from the
+    committed ncu summary, if that capture was taken of the current sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    digest = kernel_source_digest()
+    for line in open(path):
+        f = [x.strip() for x in line.strip().strip("|").split("|")]
+        if len(f) >= 3 and f[0] == w.name and f[2] == digest:
+            try:
+                return float(f[1])
+            except ValueError:
+                return None
+    return None
+
+
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
@@ -202,7 +233,14 @@ class ScanWorkload:
 
 
 class DecodeWorkload:
-    """64 successive single-token updates (one step = one token for every row)."""
+    """64 successive single-token updates (one step = one token for every row).
+
+    The state of one layer (84 MB fp32 + 10.5 MB conv state) would fit the 126 MB L2,
+    so steps rotate over LAYERS independent state buffers (one per layer of a model):
+    a step's state was last touched LAYERS - 1 steps earlier, and ~190 MB of other
+    traffic has gone through L2 since."""
+
+    LAYERS = 3
 
     def __init__(self, w, device):
         import torch
@@ -211,8 +249,10 @@ class DecodeWorkload:
         inp = synth.decode_inputs(w.batch, w.dim, w.dstate, w.steps, 4, w.dtype, seed=0)
         self.host_inp = inp
         bf = torch.bfloat16
-        self.state = torch.from_numpy(inp["state"]).to(device)
-        self.cs = torch.from_numpy(inp["conv_state"]).to(device).to(bf)
+        st = torch.from_numpy(inp["state"]).to(device)
+        cs = torch.from_numpy(inp["conv_state"]).to(device).to(bf)
+        self.states = [st.clone() for _ in range(self.LAYERS)]
+        self.css = [cs.clone() for _ in range(self.LAYERS)]
         self.seq = {k: torch.from_numpy(inp[k]).to(device).to(bf) for k in ("x", "dt", "z", "B", "C")}
         self.p = {k: torch.from_numpy(inp[k]).to(device) for k in ("A", "D", "dt_bias", "conv_w", "conv_b")}
         self.out = torch.empty(w.batch, w.dim, dtype=bf, device=device)
@@ -222,11 +262,13 @@ class DecodeWorkload:
 
     def step(self):
         s = self.k % self.w.steps
+        layer = self.k % self.LAYERS
         self.k += 1
         q, p = self.seq, self.p
-        self.ssm.ssm_selective_state_update(self.state, self.cs, q["x"][s], q["dt"][s], p["A"],
-                                            q["B"][s], q["C"][s], p["D"], q["z"][s], p["dt_bias"],
-                                            True, p["conv_w"], p["conv_b"], out=self.out)
+        self.ssm.ssm_selective_state_update(self.states[layer], self.css[layer], q["x"][s],
+                                            q["dt"][s], p["A"], q["B"][s], q["C"][s], p["D"],
+                                            q["z"][s], p["dt_bias"], True, p["conv_w"],
+                                            p["conv_b"], out=self.out)
 
     def e2e_setup(self):
         torch = self.torch
@@ -314,8 +356,13 @@ def config_of(w, args):
     if w.steps:
         c["decode_steps_cycled"] = w.steps
     ab = algorithmic_bytes(w)
-    c["l2"] = ("inputs larger than L2 ({:.0f} MB/step > 126 MB)".format(ab / 1e6)
-               if ab > L2_BYTES else "working set {:.0f} MB/step fits L2: L2-warm".format(ab / 1e6))
+    if w.name.startswith("decode"):
+        c["l2"] = (f"state rotated over {DecodeWorkload.LAYERS} layers "
+                   f"({DecodeWorkload.LAYERS * 94.5:.0f} MB of state > 126 MB L2): no step "
+                   "finds its state in L2")
+    else:
+        c["l2"] = ("inputs larger than L2 ({:.0f} MB/step > 126 MB)".format(ab / 1e6)
+                   if ab > L2_BYTES else "working set {:.0f} MB/step fits L2: L2-warm".format(ab / 1e6))
     if args.chunks:
         c["num_chunks"] = args.chunks
     return c
@@ -410,6 +457,23 @@ def main():
         exps = exp_count(w) / (w.steps if w.steps else 1) if w.name.startswith("decode") else exp_count(w)
         sfu_peak = N_SM * SFU_EX2_PER_CLK_PER_SM * sm_mhz * 1e6
         sfu_ach = exps / (mean_launch_ms * 1e-3)
+        hbm = {"achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+               "peak_kind": f"{peak_kind} HBM copy bandwidth",
+               "algorithmic_bytes_per_launch": ab}
+        sfu = {"achieved": sfu_ach / 1e9, "peak": sfu_peak / 1e9, "unit": "Gex2/s",
+               "frac": sfu_ach / sfu_peak, "exp2_per_launch": exps,
+               "peak_kind": (f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
+                             f"{sm_mhz:.0f} MHz (sampled SM clock)")}
+        traffic = recorded_traffic(w)
+        if w.name.startswith("decode"):
+            roof = dict(bound="hbm", **{k: hbm[k] for k in ("achieved", "peak", "unit", "frac")},
+                        traffic=traffic, peak_kind=hbm["peak_kind"],
+                        algorithmic_bytes_per_launch=ab, mean_launch_ms=mean_launch_ms, sfu=sfu)
+        else:
+            # one exp per (b, d, l, n) is the binding roof at d_state 16; HBM alongside
+            roof = dict(bound="alu", **{k: sfu[k] for k in ("achieved", "peak", "unit", "frac")},
+                        traffic=traffic, peak_kind=sfu["peak_kind"],
+                        exp2_per_launch=exps, mean_launch_ms=mean_launch_ms, hbm=hbm)
         line = {
             "metric": "selective-scan fwd B*D*L elems/s and achieved HBM GB/s vs B200 peak (1 GPU)",
             "value": value, "unit": "elems/s", "n_gpus": world, "steps": args.steps,
@@ -418,14 +482,8 @@ def main():
             "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic (seeded; value distributions of the Mamba init)",
             "config": config_of(w, args),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None,
-                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                         "algorithmic_bytes_per_launch": ab,
-                         "mean_launch_ms": mean_launch_ms},
-            "sfu": {"achieved": sfu_ach, "peak": sfu_peak, "unit": "ex2/s",
-                    "frac": sfu_ach / sfu_peak, "exp2_per_launch": exps,
-                    "peak_kind": f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk x {sm_mhz:.0f} MHz"},
+            "roofline": roof,
+            "hbm_gbs": achieved,
             "e2e": e2e,
             "gpu_launches": args.steps * wl.launches_per_step,
             "clocks": clocks,

@@ -14,16 +14,15 @@ namespace ssm {
 
 
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(256) conv1d_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
     using E = Elem<T>;
     constexpr int V = 8;                                  // outputs per thread
     const int L = p.seqlen;
-    const int per_row = (L + V - 1) / V;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= p.rows * per_row) return;
-    const int64_t row = gid / per_row;
-    const int t0 = (int)(gid % per_row) * V;
-    const int d = (int)(row % p.dim);
+    // grid: x = chunks of 8 outputs along the row, y = row (b, d) in slabs of 65535
+    const int t0 = (int)(blockIdx.x * blockDim.x + threadIdx.x) * V;
+    const int64_t row = (int64_t)blockIdx.z * 65535 + blockIdx.y;
+    if (t0 >= L || row >= p.rows) return;
+    const int d = (int)((uint64_t)row % (uint32_t)p.dim);
     const T* xr = static_cast<const T*>(p.x) + row * L;
     T* yr = static_cast<T*>(p.out) + row * L;
 

@@ -39,14 +39,28 @@ __device__ __forceinline__ float ex2(float x) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// softplus(x) = log(1 + e^x). Above 20 the correction log1p(e^-x) < 2.1e-9 is far
-// below fp32 resolution of x, so x itself is returned.
+// softplus(x) = log(1 + e^x) = max(x, 0) + log1p(e), e = exp(-|x|) in (0, 1].
+// log1p(e) = e * P(e) with P a degree-8 polynomial fitted by the Remez exchange
+// algorithm to log1p(e)/e on [0, 1] (max relative error 3.0e-8, below fp32's half
+// ulp), so the result keeps full relative accuracy for small e, where log(1 + e)
+// evaluated directly would lose the low bits of e. One SFU op (the exp), nine FMAs.
 __device__ __forceinline__ float softplus(float x) {
-    return x > 20.f ? x : log1pf(__expf(x));
+    const float e = ex2(-fabsf(x) * kLog2e);
+    float q = 0.00523268878685f;
+    q = fmaf(q, e, -0.029505215033f);
+    q = fmaf(q, e, 0.0782259097531f);
+    q = fmaf(q, e, -0.13663241868f);
+    q = fmaf(q, e, 0.191060047105f);
+    q = fmaf(q, e, -0.248429816251f);
+    q = fmaf(q, e, 0.33319096724f);
+    q = fmaf(q, e, -0.499994931362f);
+    q = fmaf(q, e, 0.99999996988f);
+    return fmaxf(x, 0.f) + e * q;
 }
 
-// silu(v) = v * sigmoid(v) = v / (1 + e^-v); tends to 0 for v -> -inf.
-__device__ __forceinline__ float silu(float v) { return v / (1.f + __expf(-v)); }
+// silu(v) = v * sigmoid(v) = v / (1 + e^-v): one SFU exp and one SFU reciprocal
+// (__fdividef); tends to 0 for v -> -inf (1 + e^-v overflows to inf, v / inf = 0).
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + ex2(-v * kLog2e)); }
 
 // ------------------------------------------------------ packed fp32 pairs --
 // sm_100 executes add/mul/fma on two fp32 lanes of a 64-bit register pair as one
@@ -74,6 +88,43 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
     return r;
+}
+
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 1/x on the SFU (max error about 1 ulp).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// silu on a pair of values: v / (1 + e^-v), two SFU exps and two SFU reciprocals.
+__device__ __forceinline__ uint64_t silu2(uint64_t v) {
+    const float2 f = upk2(v);
+    const uint64_t e = pk2(ex2(-f.x * kLog2e), ex2(-f.y * kLog2e));
+    const float2 den = upk2(add2(e, pk2(1.f, 1.f)));
+    return mul2(v, pk2(rcp_approx(den.x), rcp_approx(den.y)));
+}
+
+// softplus on a pair (same polynomial as softplus()).
+__device__ __forceinline__ uint64_t softplus2(uint64_t x2) {
+    const float2 x = upk2(x2);
+    const uint64_t e = pk2(ex2(-fabsf(x.x) * kLog2e), ex2(-fabsf(x.y) * kLog2e));
+    uint64_t q = pk2(0.00523268878685f, 0.00523268878685f);
+    q = fma2(q, e, pk2(-0.029505215033f, -0.029505215033f));
+    q = fma2(q, e, pk2(0.0782259097531f, 0.0782259097531f));
+    q = fma2(q, e, pk2(-0.13663241868f, -0.13663241868f));
+    q = fma2(q, e, pk2(0.191060047105f, 0.191060047105f));
+    q = fma2(q, e, pk2(-0.248429816251f, -0.248429816251f));
+    q = fma2(q, e, pk2(0.33319096724f, 0.33319096724f));
+    q = fma2(q, e, pk2(-0.499994931362f, -0.499994931362f));
+    q = fma2(q, e, pk2(0.99999996988f, 0.99999996988f));
+    return fma2(e, q, pk2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
 }
 
 // ------------------------------------------------------- shared / barriers --
@@ -123,12 +174,27 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 // exactly one translation unit (kernels.cu) includes the device headers.
 __device__ int g_device_error = 0;
 
+// try_wait with a suspend-time hint: the thread may sleep in hardware until the phase
+// completes or about `hint_ns` pass, instead of spinning and taking issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase. Returns false (and records the error) when
 // the budget runs out; the caller must then leave the kernel uniformly.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicExch(&g_device_error, 1);
             return false;
@@ -148,6 +214,33 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
+        "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 1-D bulk copy shared -> global (bulk-group completion).
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(smem_src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Order this thread's generic-proxy shared-memory writes before later async-proxy reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

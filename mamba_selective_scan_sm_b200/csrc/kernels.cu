@@ -68,24 +68,32 @@ cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps
 
 cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) {
     const int64_t per_row = (p.seqlen + 7) / 8;
-    const int64_t threads = p.rows * per_row;
-    const int64_t blocks = (threads + 255) / 256;
-    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    const unsigned bx = (unsigned)((per_row + 127) / 128);
+    const unsigned by = (unsigned)(p.rows < 65535 ? p.rows : 65535);
+    const int64_t bz = (p.rows + 65534) / 65535;
+    if (bz > 65535) return cudaErrorInvalidConfiguration;
+    const dim3 grid(bx, by, (unsigned)bz);
     if (es == 2) {
-        if (vec) conv1d_kernel<__nv_bfloat16, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else conv1d_kernel<__nv_bfloat16, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (vec) conv1d_kernel<__nv_bfloat16, true><<<grid, 128, 0, st>>>(p);
+        else conv1d_kernel<__nv_bfloat16, false><<<grid, 128, 0, st>>>(p);
     } else {
-        if (vec) conv1d_kernel<float, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else conv1d_kernel<float, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (vec) conv1d_kernel<float, true><<<grid, 128, 0, st>>>(p);
+        else conv1d_kernel<float, false><<<grid, 128, 0, st>>>(p);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_t st) {
-    // 4 lanes x 4 states covers dstate <= 16
+    if (p.bulk) {
+        const dim3 grid((unsigned)(p.dim / kDecRows), (unsigned)(p.rows / p.dim));
+        if (es == 2) decode_bulk_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
+        else decode_bulk_kernel<float><<<grid, 256, 0, st>>>(p);
+        return cudaGetLastError();
+    }
+    // 4 lanes x 4 states covers dstate <= 16; 32-bit thread indices
     const int64_t threads = p.rows * 4;
     const int64_t blocks = (threads + 255) / 256;
-    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (threads + 256 > 0x7fffffff) return cudaErrorInvalidConfiguration;
     (void)dstate;
     if (es == 2) decode_kernel<__nv_bfloat16, 4, 4><<<(unsigned)blocks, 256, 0, st>>>(p);
     else decode_kernel<float, 4, 4><<<(unsigned)blocks, 256, 0, st>>>(p);

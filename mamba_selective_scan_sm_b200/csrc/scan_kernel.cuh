@@ -33,6 +33,11 @@ namespace ssm {
 
 constexpr int kScanThreads = 128;
 
+// Steps whose state-independent operands are prepared together (a divisor of 16).
+#ifndef SSM_SCAN_BATCH
+#define SSM_SCAN_BATCH 2
+#endif
+
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 template <typename T, int NP, int S>
@@ -56,17 +61,19 @@ struct ScanCfg {
     static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, 128);
     static constexpr int STAGE = align_up(RAW_Z + G * ROWB, 1024);
     // fp32 staging
-    static constexpr int P_PITCH = TT * 8 + 8;            // float2 {delta, delta*u}
+    static constexpr int P_PITCH = TT * 8 + 16;           // float2 {delta, delta*u}; 16-B rows
     static constexpr int E_PITCH = TT * 8 + 16;           // float2 {D*u, silu(z)}
     static constexpr int OFF_P = NSTAGE * STAGE;
     static constexpr int OFF_E = OFF_P + G * P_PITCH;
     static constexpr int OFF_BT = align_up(OFF_E + G * E_PITCH, 16);
     static constexpr int OFF_CT = OFF_BT + TT * NS * 4;
-    static constexpr int OFF_PAR = OFF_CT + TT * NS * 4;  // 8 floats per channel
-    static constexpr int OFF_BAR = align_up(OFF_PAR + G * 32, 8);
+    static constexpr int OFF_PAR = OFF_CT + TT * NS * 4;  // 16 floats per channel
+    static constexpr int OFF_BAR = align_up(OFF_PAR + G * 64, 8);
     static constexpr int BYTES = OFF_BAR + NSTAGE * 8;
     static constexpr int SMEM = BYTES + 1024;             // slack for 1024-B alignment
     static_assert(TT % 16 == 0, "tile must hold whole 16-step blocks");
+    static_assert(P_PITCH % 16 == 0 && E_PITCH % 16 == 0, "staging rows take 16-byte stores");
+    static_assert(G % 2 == 0, "the prologue pairs channel rows");
     static_assert(NS <= 16, "at most 16 states");
 };
 
@@ -114,36 +121,74 @@ struct LaneState {
         if (ODD) h1 = v[NP - 1];
     }
 
-    // One time step: h = exp2(delta*a2) * h + (delta*u) * B; returns sum_k C_k h_k.
-    // bv / cv point at this lane's NP consecutive fp32 B and C values of the step.
-    __device__ __forceinline__ float step(float dl, float du, const float* bv, const float* cv) {
+    // Operands of one time step that do not depend on the state: the decay factors
+    // exp2(delta*a2), delta*u*B and C. Computing them one step ahead of the state
+    // update (software pipelining) overlaps the shared-memory loads and the SFU
+    // latency with the previous step's dependent FMAs.
+    struct In {
+        uint64_t dA[NPR > 0 ? NPR : 1], bu[NPR > 0 ? NPR : 1], cc[NPR > 0 ? NPR : 1];
+        float dA1, bu1, c1;
+    };
+
+    // pd = {delta, delta*u}; bv / cv point at this lane's NP consecutive fp32 B and C
+    // values of the step.
+    __device__ __forceinline__ In prep(const float2& pd, const float* bv, const float* cv) const {
+        In in;
+        const float dl = pd.x, du = pd.y;
         const uint64_t dd = pk2(dl, dl), uu = pk2(du, du);
+        float b[NP], cvv[NP];
+        if constexpr (NP % 4 == 0) {
+#pragma unroll
+            for (int k = 0; k < NP; k += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(bv + k);
+                b[k] = b4.x; b[k + 1] = b4.y; b[k + 2] = b4.z; b[k + 3] = b4.w;
+                if (!SUMMARY) {
+                    const float4 c4 = *reinterpret_cast<const float4*>(cv + k);
+                    cvv[k] = c4.x; cvv[k + 1] = c4.y; cvv[k + 2] = c4.z; cvv[k + 3] = c4.w;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                b[k] = bv[k];
+                if (!SUMMARY) cvv[k] = cv[k];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) {
+            const uint64_t x = mul2(dd, a2[k]);
+            in.dA[k] = pk2(ex2(lo2(x)), ex2(hi2(x)));
+            in.bu[k] = mul2(uu, pk2(b[2 * k], b[2 * k + 1]));
+            if (!SUMMARY) in.cc[k] = pk2(cvv[2 * k], cvv[2 * k + 1]);
+        }
+        if (ODD) {
+            in.dA1 = ex2(dl * a1);
+            in.bu1 = du * b[NP - 1];
+            if (!SUMMARY) in.c1 = cvv[NP - 1];
+        }
+        return in;
+    }
+
+    // h = dA * h + delta*u*B; returns sum_k C_k h_k (SUMMARY: accumulates prod dA).
+    __device__ __forceinline__ float update(const In& in) {
         uint64_t s = pk2(0.f, 0.f);
         float s1 = 0.f;
 #pragma unroll
         for (int k = 0; k < NPR; ++k) {
-            const float2 bb = *reinterpret_cast<const float2*>(bv + 2 * k);
-            const uint64_t x = mul2(dd, a2[k]);
-            const uint64_t dA = pk2(ex2(lo2(x)), ex2(hi2(x)));
-            h2[k] = fma2(dA, h2[k], mul2(uu, pk2(bb.x, bb.y)));
-            if (SUMMARY) {
-                pr2[k] = mul2(pr2[k], dA);
-            } else {
-                const float2 cc = *reinterpret_cast<const float2*>(cv + 2 * k);
-                s = fma2(pk2(cc.x, cc.y), h2[k], s);
-            }
+            h2[k] = fma2(in.dA[k], h2[k], in.bu[k]);
+            if (SUMMARY) pr2[k] = mul2(pr2[k], in.dA[k]);
+            else s = (k == 0) ? mul2(in.cc[k], h2[k]) : fma2(in.cc[k], h2[k], s);
         }
         if (ODD) {
-            const float dA = ex2(dl * a1);
-            h1 = fmaf(dA, h1, du * bv[NP - 1]);
-            if (SUMMARY) pr1 *= dA;
-            else s1 = cv[NP - 1] * h1;
+            h1 = fmaf(in.dA1, h1, in.bu1);
+            if (SUMMARY) pr1 *= in.dA1;
+            else s1 = in.c1 * h1;
         }
+        if (SUMMARY) return 0.f;
         return (NPR > 0 ? lo2(s) + hi2(s) : 0.f) + s1;
     }
 };
 
-// At most 128 registers per thread, so four 128-thread CTAs fit an SM's register file.
 template <typename T, int NP, int S, bool USE_TMA, bool SUMMARY>
 __global__ void __launch_bounds__(kScanThreads, 4)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
@@ -251,21 +296,24 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    // Per-direction channel parameters -> smem (8 floats per channel slot).
+    // Per-direction channel parameters -> smem, 16 floats per channel slot, each value
+    // stored twice so a 64-bit load yields the pair the packed prologue math needs:
+    // {w0,w0, w1,w1, w2,w2, w3,w3, conv_b x2, dt_bias x2, D x2, 0, 0}.
     auto load_params = [&](int dir) {
         for (int e = tid; e < G; e += kScanThreads) {
             const int dd = d0 + e;
-            float* q = par + e * 8;
+            float* q = par + e * 16;
             const bool ok = dd < p.dim;
-            // conv taps right-aligned: q[3] meets the newest input
+            // conv taps right-aligned: tap 3 meets the newest input
             for (int k = 0; k < 4; ++k) {
                 const int kk = k - (4 - p.conv_width);
-                q[k] = (ok && conv && kk >= 0) ? p.conv_w[(int64_t)dd * p.conv_width + kk] : 0.f;
+                q[2 * k] = q[2 * k + 1] =
+                    (ok && conv && kk >= 0) ? p.conv_w[(int64_t)dd * p.conv_width + kk] : 0.f;
             }
-            q[4] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
-            q[5] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
-            q[6] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
-            q[7] = 0.f;
+            q[8] = q[9] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
+            q[10] = q[11] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
+            q[12] = q[13] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
+            q[14] = q[15] = 0.f;
         }
     };
 
@@ -315,36 +363,43 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll
             for (int m = 0; m < EPC; ++m) dst[m * NS] = E::to_f(tv[m]);
         }
-        // per (channel, t) quantities; a warp walks one channel row, lanes along t
-        for (int idx = warp; idx < G * (TT / 32); idx += kScanThreads / 32) {
-            const int r = idx / (TT / 32);
-            const int tt = (idx % (TT / 32)) * 32 + lane;
+        // per (channel, t) quantities, two consecutive steps per lane in packed pairs:
+        // 16 lanes cover one 32-step channel row, a warp two rows at a time
+        for (int idx = warp; idx < G / 2; idx += kScanThreads / 32) {
+            const int r = 2 * idx + (lane >> 4);
+            const int tt = 2 * (lane & 15);                 // steps tt and tt + 1
             const T* xr = reinterpret_cast<const T*>(st + Cfg::RAW_X + r * xpitch);
-            const float* q = par + r * 8;
-            float u;
+            const uint64_t* q2 = reinterpret_cast<const uint64_t*>(par + r * 16);
+            uint64_t u2;
             if (conv) {
-                float acc = q[4];
-                if (!rv) {
+                // forward: u_t = sum_k w_k x[t-3+k]; reverse: u_t = sum_k w_k x[t+3-k]
+                float xv[5];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) acc = fmaf(q[k], E::to_f(xr[xoff + tt - 3 + k]), acc);
-                } else {
+                for (int m = 0; m < 5; ++m)
+                    xv[m] = E::to_f(rv ? xr[tt + 4 - m] : xr[xoff + tt - 3 + m]);
+                uint64_t acc = q2[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) acc = fmaf(q[k], E::to_f(xr[tt + 3 - k]), acc);
-                }
-                u = silu(acc);
+                for (int k = 0; k < 4; ++k)
+                    acc = fma2(q2[k], rv ? pk2(xv[k + 1], xv[k]) : pk2(xv[k], xv[k + 1]), acc);
+                u2 = silu2(acc);
             } else {
-                u = E::to_f(xr[tt]);
+                u2 = pk2(E::to_f(xr[tt]), E::to_f(xr[tt + 1]));
             }
-            float dl = E::to_f(reinterpret_cast<const T*>(st + Cfg::RAW_DT)[r * TT + tt]) + q[5];
-            if (p.softplus) dl = softplus(dl);
-            reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(Pbuf) + r * Cfg::P_PITCH)[tt] =
-                make_float2(dl, dl * u);
+            const T* dtr = reinterpret_cast<const T*>(st + Cfg::RAW_DT) + r * TT + tt;
+            uint64_t dl2 = add2(pk2(E::to_f(dtr[0]), E::to_f(dtr[1])), q2[5]);
+            if (p.softplus) dl2 = softplus2(dl2);
+            const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
+            *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(Pbuf) + r * Cfg::P_PITCH + tt * 8) =
+                make_float4(dl.x, du.x, dl.y, du.y);
             if (!SUMMARY) {
-                const float g =
-                    has_z ? silu(E::to_f(reinterpret_cast<const T*>(st + Cfg::RAW_Z)[r * TT + tt]))
-                          : 1.f;
-                reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(Ebuf) + r * Cfg::E_PITCH)[tt] =
-                    make_float2(q[6] * u, g);
+                uint64_t g2 = pk2(1.f, 1.f);
+                if (has_z) {
+                    const T* zr = reinterpret_cast<const T*>(st + Cfg::RAW_Z) + r * TT + tt;
+                    g2 = silu2(pk2(E::to_f(zr[0]), E::to_f(zr[1])));
+                }
+                const float2 g = upk2(g2), dv = upk2(mul2(q2[6], u2));
+                *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(Ebuf) + r * Cfg::E_PITCH + tt * 8) =
+                    make_float4(dv.x, g.x, dv.y, g.y);
             }
         }
     };
@@ -452,14 +507,29 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         for (int blk = 0; blk < TT / 16; ++blk) {
             if (!FULL && blk * 16 >= nvalid) break;
             float acc[16];
+            if (FULL) {
+                // K steps at a time: their state-independent operands (shared-memory
+                // loads, delta*A, the SFU exps, delta*u*B) are all prepared first, as K
+                // independent streams, then the K dependent state updates run.
+                constexpr int K = SSM_SCAN_BATCH;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int ii = blk * 16 + q;
-                const int tt = RV ? TT - 1 - ii : ii;
-                acc[q] = 0.f;
-                if (FULL || ii < nvalid) {
-                    const float2 pd = Prow[tt];
-                    acc[q] = ls.step(pd.x, pd.y, Bl + tt * NS, Cl + tt * NS);
+                for (int q0 = 0; q0 < 16; q0 += K) {
+                    typename LaneState<NP, SUMMARY>::In in[K];
+#pragma unroll
+                    for (int u = 0; u < K; ++u) {
+                        const int tt = RV ? TT - 1 - (blk * 16 + q0 + u) : blk * 16 + q0 + u;
+                        in[u] = ls.prep(Prow[tt], Bl + tt * NS, Cl + tt * NS);
+                    }
+#pragma unroll
+                    for (int u = 0; u < K; ++u) acc[q0 + u] = ls.update(in[u]);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int ii = blk * 16 + q;
+                    const int tt = RV ? TT - 1 - ii : ii;
+                    acc[q] = 0.f;
+                    if (ii < nvalid) acc[q] = ls.update(ls.prep(Prow[tt], Bl + tt * NS, Cl + tt * NS));
                 }
             }
             if (SUMMARY) continue;
@@ -508,7 +578,12 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         bool ok = true;
         const uint8_t* st;
         if (USE_TMA) {
-            ok = mbar_wait_bounded(&bars[f % NSTAGE], (f / NSTAGE) & 1);
+            // one lane per warp polls; __syncwarp hands the completed phase to the rest
+            if (lane == 0) ok = mbar_wait_bounded(&bars[f % NSTAGE], (f / NSTAGE) & 1);
+            __syncwarp();
+            // each lane then observes the completed phase itself (one try_wait, which
+            // succeeds at once), so the TMA writes are acquired by every reader
+            if (lane != 0) mbar_try_wait(&bars[f % NSTAGE], (f / NSTAGE) & 1);
             st = smem + (f % NSTAGE) * Cfg::STAGE;
         } else {
             load_plain(f);

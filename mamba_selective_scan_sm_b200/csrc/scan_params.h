@@ -67,6 +67,7 @@ struct DecodeParams {
     int64_t rows;       // batch * dim
     int dim, dstate, conv_width, softplus;
     int vec;            // dstate == 16 and state / A rows 16-byte aligned
+    int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
 };
 
 }  // namespace ssm

@@ -362,6 +362,8 @@ ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const vo
     if (dim > 0x3fffffffLL) return fail(SSM_ERR_BAD_SHAPE, "dim must be below 2^30");
     const int64_t rows = batch * dim;
     if (rows == 0) return ok();
+    if (rows > (int64_t)1 << 28)
+        return fail(SSM_ERR_BAD_SHAPE, "batch * dim = %lld exceeds 2^28", (long long)rows);
     struct { const void* p; const char* n; } req[] = {
         {state, "state"}, {x, "x"}, {dt, "dt"}, {A, "A"}, {B_t, "B_t"}, {C_t, "C_t"}, {out, "out"}};
     for (auto& r : req)
@@ -400,6 +402,10 @@ ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const vo
     p.conv_width = conv_weight ? conv_width : 0;
     p.softplus = dt_softplus ? 1 : 0;
     p.vec = dstate == 16 && aligned(state, 16) && aligned(A, 16);
+    // bulk-copy variant: 64-row groups of 16-byte aligned rows
+    p.bulk = dim % 64 == 0 && batch <= 65535 && aligned(state, 16) && aligned(x, 16) && aligned(dt, 16) &&
+             aligned(out, 16) && (!z || aligned(z, 16)) &&
+             (!conv_weight || aligned(conv_state, 16)) && env_int("SSM_DECODE_PLAIN", 0) == 0;
     cudaError_t e = ssm::launch_decode(es, (int)dstate, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return ok();

@@ -148,3 +148,33 @@ def test_decode_repeated_equals_scan_on_gpu(dtype):
     else:
         assert_close(host(yd), host(y), dtype, "decode^L vs scan")
     state_close(host(st), host(h), "state")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dstate", [16, 5])
+@pytest.mark.parametrize("width", [4, 2, 3])
+@pytest.mark.parametrize("opts", [dict(), dict(conv=False), dict(gate=False, skip=False)],
+                         ids=["full", "no-conv", "no-z-no-D"])
+def test_decode_bulk_path_matches_oracle(dtype, dstate, width, opts):
+    """Rows a multiple of 64 with 16-byte aligned bases take the bulk-copy kernel."""
+    B, D, steps = 2, 96, 6                       # 192 rows = 3 bulk groups
+    inp = synth.decode_inputs(B, D, dstate, steps, width, dtype, seed=27)
+    yg, sg, cg = _decode_gpu(inp, dtype, steps, **opts)
+    yo, so, co = _decode_oracle(inp, steps, **opts)
+    for s in range(steps):
+        assert_close_out(yg[s], yo[s], dtype, f"y step {s}")
+    state_close(sg, so, "state")
+    if opts.get("conv", True):
+        np.testing.assert_array_equal(cg, co)
+
+
+def test_decode_bulk_and_plain_paths_agree(monkeypatch):
+    B, D, steps = 2, 128, 4
+    inp = synth.decode_inputs(B, D, 16, steps, 4, "bf16", seed=28)
+    yb, sb, cb = _decode_gpu(inp, "bf16", steps)
+    monkeypatch.setenv("SSM_DECODE_PLAIN", "1")
+    yp, sp, cp = _decode_gpu(inp, "bf16", steps)
+    for s in range(steps):
+        assert_bf16_ulp(yb[s], yp[s], f"step {s}")
+    state_close(sb, sp, "state")
+    np.testing.assert_array_equal(cb, cp)
