@@ -9,45 +9,48 @@ namespace ssm {
 
 namespace {
 
-template <typename T, int NP, int S>
+template <typename T, int NP, int S, int KC>
 ScanVariant variant_of() {
-    using Cfg = ScanCfg<T, NP, S>;
-    return ScanVariant{(int)sizeof(T), NP, S, Cfg::G, Cfg::TT, Cfg::HALO, Cfg::SMEM};
+    using Cfg = ScanCfg<T, NP, S, KC>;
+    return ScanVariant{(int)sizeof(T), NP, S, KC, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM};
 }
 
-template <typename T, int NP, int S, bool TMA, bool SUM>
+template <typename T, int NP, int S, int KC, bool TMA, bool SUM>
 cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
-    using Cfg = ScanCfg<T, NP, S>;
-    auto* k = scan_fwd_kernel<T, NP, S, TMA, SUM>;
+    using Cfg = ScanCfg<T, NP, S, KC>;
+    auto* k = scan_fwd_kernel<T, NP, S, KC, TMA, SUM>;
     static const cudaError_t attr =
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (attr != cudaSuccess) return attr;
-    k<<<grid, kScanThreads, Cfg::SMEM, st>>>(maps, p);
+    k<<<grid, Cfg::NT, Cfg::SMEM, st>>>(maps, p);
     return cudaGetLastError();
 }
 
-template <typename T, int NP, int S>
+template <typename T, int NP, int S, int KC>
 cudaError_t launch_t(bool tma, bool sum, const ScanMaps& maps, const ScanParams& p, dim3 grid,
                      cudaStream_t st) {
-    if (tma) return sum ? launch_one<T, NP, S, true, true>(maps, p, grid, st)
-                        : launch_one<T, NP, S, true, false>(maps, p, grid, st);
-    return sum ? launch_one<T, NP, S, false, true>(maps, p, grid, st)
-               : launch_one<T, NP, S, false, false>(maps, p, grid, st);
+    if (tma) return sum ? launch_one<T, NP, S, KC, true, true>(maps, p, grid, st)
+                        : launch_one<T, NP, S, KC, true, false>(maps, p, grid, st);
+    return sum ? launch_one<T, NP, S, KC, false, true>(maps, p, grid, st)
+               : launch_one<T, NP, S, KC, false, false>(maps, p, grid, st);
 }
 
 }  // namespace
 
+// (states per lane, lanes per channel, channels per lane)
 #define SSM_SCAN_VARIANTS(X) \
-    X(4, 4)                  \
-    X(2, 8)                  \
-    X(2, 4)                  \
-    X(1, 4)
+    X(4, 4, 1)               \
+    X(4, 4, 2)               \
+    X(2, 8, 1)               \
+    X(2, 8, 2)               \
+    X(2, 4, 1)               \
+    X(1, 4, 1)
 
-bool scan_variant(int es, int np, int s, ScanVariant* v) {
-#define X(NP_, S_)                                                          \
-    if (np == NP_ && s == S_) {                                             \
-        *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_>()                 \
-                     : variant_of<float, NP_, S_>();                        \
+bool scan_variant(int es, int np, int s, int kc, ScanVariant* v) {
+#define X(NP_, S_, KC_)                                                     \
+    if (np == NP_ && s == S_ && kc == KC_) {                                \
+        *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_, KC_>()            \
+                     : variant_of<float, NP_, S_, KC_>();                   \
         return es == 2 || es == 4;                                          \
     }
     SSM_SCAN_VARIANTS(X)
@@ -57,10 +60,11 @@ bool scan_variant(int es, int np, int s, ScanVariant* v) {
 
 cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
                         const ScanParams& p, dim3 grid, cudaStream_t st) {
-#define X(NP_, S_)                                                                    \
-    if (v.np == NP_ && v.s == S_)                                                     \
-        return v.elem_size == 2 ? launch_t<__nv_bfloat16, NP_, S_>(tma, sum, maps, p, grid, st) \
-                                : launch_t<float, NP_, S_>(tma, sum, maps, p, grid, st);
+#define X(NP_, S_, KC_)                                                                   \
+    if (v.np == NP_ && v.s == S_ && v.kc == KC_)                                          \
+        return v.elem_size == 2                                                           \
+                   ? launch_t<__nv_bfloat16, NP_, S_, KC_>(tma, sum, maps, p, grid, st)   \
+                   : launch_t<float, NP_, S_, KC_>(tma, sum, maps, p, grid, st);
     SSM_SCAN_VARIANTS(X)
 #undef X
     return cudaErrorInvalidValue;

@@ -12,14 +12,16 @@ struct ScanVariant {
     int elem_size;      // 2 (bf16) or 4 (fp32)
     int np;             // states per lane
     int s;              // lanes per channel
-    int channels;       // channels per CTA (128 / s)
+    int kc;             // channels per lane
+    int channels;       // channels per CTA
+    int threads;        // threads per CTA
     int tile;           // time steps per tile (128 bytes of elements)
     int halo;           // conv history elements fetched with a tile
     int smem_bytes;     // dynamic shared memory per CTA
 };
 
-// Returns false if (elem_size, np, s) has no compiled kernel.
-bool scan_variant(int elem_size, int np, int s, ScanVariant* v);
+// Returns false if (elem_size, np, s, kc) has no compiled kernel.
+bool scan_variant(int elem_size, int np, int s, int kc, ScanVariant* v);
 
 cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, const ScanMaps& maps,
                         const ScanParams& p, dim3 grid, cudaStream_t stream);

@@ -31,8 +31,6 @@
 
 namespace ssm {
 
-constexpr int kScanThreads = 128;
-
 // Steps whose state-independent operands are prepared together (a divisor of 16).
 #ifndef SSM_SCAN_BATCH
 #define SSM_SCAN_BATCH 2
@@ -40,10 +38,10 @@ constexpr int kScanThreads = 128;
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <typename T, int NP, int S>
+template <typename T, int NP, int S, int KC>
 struct ScanCfg {
-    static constexpr int NT = kScanThreads;
-    static constexpr int G = NT / S;          // channels per CTA
+    static constexpr int G = S == 4 ? 32 : 16;          // channels per CTA
+    static constexpr int NT = G * S / KC;               // threads per CTA
     static constexpr int NS = NP * S;         // padded state count
     static constexpr int ES = sizeof(T);
     static constexpr int TT = 32;             // tile length (time steps)
@@ -60,14 +58,17 @@ struct ScanCfg {
     static constexpr int RAW_DT = align_up(RAW_X + G * X_PITCH_MAX, 128);
     static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, 128);
     static constexpr int STAGE = align_up(RAW_Z + G * ROWB, 1024);
-    // fp32 staging
-    static constexpr int P_PITCH = TT * 8 + 16;           // float2 {delta, delta*u}; 16-B rows
-    static constexpr int E_PITCH = TT * 8 + 16;           // float2 {D*u, silu(z)}
+    // fp32 staging. P: per channel group of KC channels and step, KC x {delta, delta*u}.
+    static constexpr int P_PITCH = TT * KC * 8 + 16;
+    static constexpr int E_PITCH = TT * 8 + 16;           // per channel: {D*u, silu(z)}
     static constexpr int OFF_P = NSTAGE * STAGE;
-    static constexpr int OFF_E = OFF_P + G * P_PITCH;
+    static constexpr int OFF_E = OFF_P + (G / KC) * P_PITCH;
+    // Transposed B, C: [t][n] in the input type (bf16 stays bf16: exact, and half the
+    // shared-memory bytes each lane reads per step; fp32 stays fp32).
+    static constexpr int BCS = ES;
     static constexpr int OFF_BT = align_up(OFF_E + G * E_PITCH, 16);
-    static constexpr int OFF_CT = OFF_BT + TT * NS * 4;
-    static constexpr int OFF_PAR = OFF_CT + TT * NS * 4;  // 16 floats per channel
+    static constexpr int OFF_CT = OFF_BT + TT * NS * BCS;
+    static constexpr int OFF_PAR = align_up(OFF_CT + TT * NS * BCS, 16);  // 16 floats per channel
     static constexpr int OFF_BAR = align_up(OFF_PAR + G * 64, 8);
     static constexpr int BYTES = OFF_BAR + NSTAGE * 8;
     static constexpr int SMEM = BYTES + 1024;             // slack for 1024-B alignment
@@ -75,6 +76,7 @@ struct ScanCfg {
     static_assert(P_PITCH % 16 == 0 && E_PITCH % 16 == 0, "staging rows take 16-byte stores");
     static_assert(G % 2 == 0, "the prologue pairs channel rows");
     static_assert(NS <= 16, "at most 16 states");
+    static_assert(KC == 1 || KC == 2, "one or two channels per lane");
 };
 
 // Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 128-B
@@ -130,30 +132,10 @@ struct LaneState {
         float dA1, bu1, c1;
     };
 
-    // pd = {delta, delta*u}; bv / cv point at this lane's NP consecutive fp32 B and C
-    // values of the step.
-    __device__ __forceinline__ In prep(const float2& pd, const float* bv, const float* cv) const {
+    // dl = delta, du = delta*u of the step; b / cvv: this lane's NP fp32 B and C values.
+    __device__ __forceinline__ In prep(float dl, float du, const float* b, const float* cvv) const {
         In in;
-        const float dl = pd.x, du = pd.y;
         const uint64_t dd = pk2(dl, dl), uu = pk2(du, du);
-        float b[NP], cvv[NP];
-        if constexpr (NP % 4 == 0) {
-#pragma unroll
-            for (int k = 0; k < NP; k += 4) {
-                const float4 b4 = *reinterpret_cast<const float4*>(bv + k);
-                b[k] = b4.x; b[k + 1] = b4.y; b[k + 2] = b4.z; b[k + 3] = b4.w;
-                if (!SUMMARY) {
-                    const float4 c4 = *reinterpret_cast<const float4*>(cv + k);
-                    cvv[k] = c4.x; cvv[k + 1] = c4.y; cvv[k + 2] = c4.z; cvv[k + 3] = c4.w;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                b[k] = bv[k];
-                if (!SUMMARY) cvv[k] = cv[k];
-            }
-        }
 #pragma unroll
         for (int k = 0; k < NPR; ++k) {
             const uint64_t x = mul2(dd, a2[k]);
@@ -189,10 +171,13 @@ struct LaneState {
     }
 };
 
-template <typename T, int NP, int S, bool USE_TMA, bool SUMMARY>
-__global__ void __launch_bounds__(kScanThreads, 4)
+// Four CTAs per SM at least: 128 registers per thread with 128-thread CTAs, up to
+// 255 with the 64-thread CTAs of the two-channel variant (shared memory allows 5).
+template <typename T, int NP, int S, int KC, bool USE_TMA, bool SUMMARY>
+__global__ void __launch_bounds__(ScanCfg<T, NP, S, KC>::NT, 4)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
-    using Cfg = ScanCfg<T, NP, S>;
+    using Cfg = ScanCfg<T, NP, S, KC>;
+    constexpr int NT = Cfg::NT;
     using E = Elem<T>;
     constexpr int G = Cfg::G, NS = Cfg::NS, TT = Cfg::TT, HALO = Cfg::HALO, R = Cfg::R;
     constexpr int ROWB = Cfg::ROWB, SWZ = Cfg::SWZ;
@@ -203,19 +188,17 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     float2* Pbuf = reinterpret_cast<float2*>(smem + Cfg::OFF_P);
     float2* Ebuf = reinterpret_cast<float2*>(smem + Cfg::OFF_E);
-    float* Bt = reinterpret_cast<float*>(smem + Cfg::OFF_BT);
-    float* Ct = reinterpret_cast<float*>(smem + Cfg::OFF_CT);
+    T* Bt = reinterpret_cast<T*>(smem + Cfg::OFF_BT);
+    T* Ct = reinterpret_cast<T*>(smem + Cfg::OFF_CT);
     float* par = reinterpret_cast<float*>(smem + Cfg::OFF_PAR);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int c = tid / S;          // channel slot in the CTA
+    const int lg = tid / S;         // lane group: channels lg*KC .. lg*KC + KC - 1 of the CTA
     const int j = tid % S;          // state group of this lane
     const int b = blockIdx.y;
     const int d0 = blockIdx.x * G;
-    const int d = d0 + c;
-    const bool dvalid = d < p.dim;
     const int L = p.seqlen;
     const int chunk = blockIdx.z;
     const int cs = chunk * p.chunk_len;                    // first scan position
@@ -226,7 +209,8 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     const bool has_z = !SUMMARY && p.z != nullptr;
     const bool conv = p.conv_w != nullptr;
     const int xpitch = conv ? Cfg::X_PITCH_MAX : TT * (int)sizeof(T);
-    const int64_t row = (int64_t)b * p.dim + d;           // (b, d) row index
+    auto chan_d = [&](int k) { return d0 + lg * KC + k; };             // channel k of the lane
+    auto chan_row = [&](int k) { return (int64_t)b * p.dim + chan_d(k); };  // its (b, d) row
 
     auto tile_rev = [&](int f) { return p.mode == 1 || (p.mode == 2 && f >= ntl); };
     // time of the first element of flat tile f
@@ -268,7 +252,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         const bool rv = tile_rev(f);
         const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
         const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
-        for (int e = tid; e < NS * TT; e += kScanThreads) {
+        for (int e = tid; e < NS * TT; e += NT) {
             const int n = e / TT, col = e % TT, t = l0 + col;
             const bool ok = n < p.dstate && t >= 0 && t < L;
             const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
@@ -277,14 +261,14 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
         const int xw = xpitch / (int)sizeof(T);
         const int xs = (conv && !rv) ? l0 - HALO : l0;
-        for (int e = tid; e < G * xw; e += kScanThreads) {
+        for (int e = tid; e < G * xw; e += NT) {
             const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
             const bool ok = dd < p.dim && t >= 0 && t < L;
             const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
             reinterpret_cast<T*>(st + Cfg::RAW_X + r * xpitch)[col] =
                 ok ? static_cast<const T*>(p.u)[gi] : T(0.f);
         }
-        for (int e = tid; e < G * TT; e += kScanThreads) {
+        for (int e = tid; e < G * TT; e += NT) {
             const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
             const bool ok = dd < p.dim && t >= 0 && t < L;
             const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
@@ -300,7 +284,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     // stored twice so a 64-bit load yields the pair the packed prologue math needs:
     // {w0,w0, w1,w1, w2,w2, w3,w3, conv_b x2, dt_bias x2, D x2, 0, 0}.
     auto load_params = [&](int dir) {
-        for (int e = tid; e < G; e += kScanThreads) {
+        for (int e = tid; e < G; e += NT) {
             const int dd = d0 + e;
             float* q = par + e * 16;
             const bool ok = dd < p.dim;
@@ -317,55 +301,63 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    LaneState<NP, SUMMARY> ls;
+    LaneState<NP, SUMMARY> ls[KC];
     auto load_A = [&](int dir) {
-        float a[NP];
 #pragma unroll
-        for (int k = 0; k < NP; ++k) {
-            const int n = j * NP + k;
-            a[k] = (dvalid && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
+        for (int k = 0; k < KC; ++k) {
+            const int d = chan_d(k);
+            float a[NP];
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                const int n = j * NP + i;
+                a[i] = (d < p.dim && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e
+                                                   : 0.f;
+            }
+            ls[k].set_a(a);
         }
-        ls.set_a(a);
     };
     // Initial state of this chunk: carry over the summaries of earlier chunks.
     auto init_state = [&]() {
-        ls.reset();
-        if (!SUMMARY && chunk > 0 && dvalid) {
-            float hv[NP];
 #pragma unroll
-            for (int k = 0; k < NP; ++k) hv[k] = 0.f;
-            const int64_t stride = (int64_t)p.batch * p.dim * NS;
-            for (int k2 = 0; k2 < chunk; ++k2) {
-                const float2* sm = p.summary + k2 * stride + row * NS + j * NP;
+        for (int k = 0; k < KC; ++k) {
+            ls[k].reset();
+            if (!SUMMARY && chunk > 0 && chan_d(k) < p.dim) {
+                float hv[NP];
 #pragma unroll
-                for (int k = 0; k < NP; ++k) {
-                    const float2 ps = sm[k];
-                    hv[k] = fmaf(ps.x, hv[k], ps.y);
+                for (int i = 0; i < NP; ++i) hv[i] = 0.f;
+                const int64_t stride = (int64_t)p.batch * p.dim * NS;
+                for (int k2 = 0; k2 < chunk; ++k2) {
+                    const float2* sm = p.summary + k2 * stride + chan_row(k) * NS + j * NP;
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) {
+                        const float2 ps = sm[i];
+                        hv[i] = fmaf(ps.x, hv[i], ps.y);
+                    }
                 }
+                ls[k].set(hv);
             }
-            ls.set(hv);
         }
     };
 
     auto prologue = [&](int f, const uint8_t* st) {
         const bool rv = tile_rev(f);
         const int xoff = (conv && !rv) ? HALO : 0;
-        // B, C: swizzled [n][t] (input dtype) -> [t][n] fp32, one 16-byte chunk per thread
+        // B, C: swizzled [n][t] -> [t][n] in the input type, one 16-byte chunk per thread
         constexpr int EPC = 16 / (int)sizeof(T);           // elements per 16-byte chunk
         constexpr int NCH = NS * ROWB / 16;                // chunks per tensor
-        for (int e = tid; e < 2 * NCH; e += kScanThreads) {
+        for (int e = tid; e < 2 * NCH; e += NT) {
             const int ten = e / NCH, ch = e % NCH;
             const int n = ch % NS, t0 = (ch / NS) * EPC;
             const uint8_t* src = st + (ten ? Cfg::RAW_C : Cfg::RAW_B) + swz<ROWB, SWZ>(n, t0 * (int)sizeof(T));
-            float* dst = (ten ? Ct : Bt) + t0 * NS + n;
+            T* dst = (ten ? Ct : Bt) + t0 * NS + n;
             const uint4 v = *reinterpret_cast<const uint4*>(src);
             const T* tv = reinterpret_cast<const T*>(&v);
 #pragma unroll
-            for (int m = 0; m < EPC; ++m) dst[m * NS] = E::to_f(tv[m]);
+            for (int m = 0; m < EPC; ++m) dst[m * NS] = tv[m];
         }
         // per (channel, t) quantities, two consecutive steps per lane in packed pairs:
         // 16 lanes cover one 32-step channel row, a warp two rows at a time
-        for (int idx = warp; idx < G / 2; idx += kScanThreads / 32) {
+        for (int idx = warp; idx < G / 2; idx += NT / 32) {
             const int r = 2 * idx + (lane >> 4);
             const int tt = 2 * (lane & 15);                 // steps tt and tt + 1
             const T* xr = reinterpret_cast<const T*>(st + Cfg::RAW_X + r * xpitch);
@@ -389,8 +381,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             uint64_t dl2 = add2(pk2(E::to_f(dtr[0]), E::to_f(dtr[1])), q2[5]);
             if (p.softplus) dl2 = softplus2(dl2);
             const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
-            *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(Pbuf) + r * Cfg::P_PITCH + tt * 8) =
-                make_float4(dl.x, du.x, dl.y, du.y);
+            uint8_t* prow = reinterpret_cast<uint8_t*>(Pbuf) + (r / KC) * Cfg::P_PITCH;
+            if (KC == 1) {
+                *reinterpret_cast<float4*>(prow + tt * 8) = make_float4(dl.x, du.x, dl.y, du.y);
+            } else {
+                *reinterpret_cast<float2*>(prow + tt * 16 + (r % KC) * 8) = make_float2(dl.x, du.x);
+                *reinterpret_cast<float2*>(prow + tt * 16 + 16 + (r % KC) * 8) = make_float2(dl.y, du.y);
+            }
             if (!SUMMARY) {
                 uint64_t g2 = pk2(1.f, 1.f);
                 if (has_z) {
@@ -404,15 +401,78 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    const float2* Prow = reinterpret_cast<const float2*>(reinterpret_cast<uint8_t*>(Pbuf) +
-                                                          c * Cfg::P_PITCH);
-    const float2* Erow = reinterpret_cast<const float2*>(reinterpret_cast<uint8_t*>(Ebuf) +
-                                                          c * Cfg::E_PITCH);
-    const float* Bl = Bt + j * NP;
-    const float* Cl = Ct + j * NP;
-
+    const uint8_t* Prow = reinterpret_cast<uint8_t*>(Pbuf) + lg * Cfg::P_PITCH;
+    const T* Bl = Bt + j * NP;
+    const T* Cl = Ct + j * NP;
+    // P of step tt for the lane's KC channels: pd[k] = {delta, delta*u}
+    auto load_p = [&](int tt, float2 (&pd)[KC]) {
+        if constexpr (KC == 2) {
+            const float4 v = *reinterpret_cast<const float4*>(Prow + tt * 16);
+            pd[0] = make_float2(v.x, v.y);
+            pd[1] = make_float2(v.z, v.w);
+        } else {
+            pd[0] = *reinterpret_cast<const float2*>(Prow + tt * 8);
+        }
+    };
+    // this lane's NP values of B and C at step tt (bf16 pairs are widened in registers:
+    // the high half of a 32-bit word is already an fp32 bit pattern, the low half
+    // shifted up by 16 is one)
+    auto load_bc = [&](int tt, float (&bv)[NP], float (&cv)[NP]) {
+        if constexpr (sizeof(T) == 2 && NP % 2 == 0) {
+            uint32_t wb[NP / 2], wc[NP / 2];
+            if constexpr (NP == 4) {
+                const uint2 b2 = *reinterpret_cast<const uint2*>(Bl + tt * NS);
+                wb[0] = b2.x; wb[1] = b2.y;
+                if (!SUMMARY) {
+                    const uint2 c2 = *reinterpret_cast<const uint2*>(Cl + tt * NS);
+                    wc[0] = c2.x; wc[1] = c2.y;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < NP / 2; ++i) {
+                    wb[i] = reinterpret_cast<const uint32_t*>(Bl + tt * NS)[i];
+                    if (!SUMMARY) wc[i] = reinterpret_cast<const uint32_t*>(Cl + tt * NS)[i];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < NP / 2; ++i) {
+                bv[2 * i] = __uint_as_float(wb[i] << 16);
+                bv[2 * i + 1] = __uint_as_float(wb[i] & 0xffff0000u);
+                if (!SUMMARY) {
+                    cv[2 * i] = __uint_as_float(wc[i] << 16);
+                    cv[2 * i + 1] = __uint_as_float(wc[i] & 0xffff0000u);
+                }
+            }
+        } else if constexpr (sizeof(T) == 4 && NP % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < NP; i += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(Bl + tt * NS + i);
+                bv[i] = b4.x; bv[i + 1] = b4.y; bv[i + 2] = b4.z; bv[i + 3] = b4.w;
+                if (!SUMMARY) {
+                    const float4 c4 = *reinterpret_cast<const float4*>(Cl + tt * NS + i);
+                    cv[i] = c4.x; cv[i + 1] = c4.y; cv[i + 2] = c4.z; cv[i + 3] = c4.w;
+                }
+            }
+        } else if constexpr (sizeof(T) == 4 && NP == 2) {
+            const float2 b2 = *reinterpret_cast<const float2*>(Bl + tt * NS);
+            bv[0] = b2.x; bv[1] = b2.y;
+            if (!SUMMARY) {
+                const float2 c2 = *reinterpret_cast<const float2*>(Cl + tt * NS);
+                cv[0] = c2.x; cv[1] = c2.y;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NP; ++i) {
+                bv[i] = E::to_f(Bl[tt * NS + i]);
+                if (!SUMMARY) cv[i] = E::to_f(Cl[tt * NS + i]);
+            }
+        }
+    };
     // gate, skip term, bidirectional partial and the store of R owned outputs
-    auto epilogue = [&](const float* acc, bool rv, int dir, int l0, int pos0, int nown) {
+    auto epilogue = [&](int k, const float* acc, bool rv, int dir, int l0, int pos0, int nown) {
+        const float2* Erow = reinterpret_cast<const float2*>(
+            reinterpret_cast<uint8_t*>(Ebuf) + (lg * KC + k) * Cfg::E_PITCH);
+        const int64_t row = chan_row(k);
         float yv[R];
 #pragma unroll
         for (int m = 0; m < R; ++m) {
@@ -421,7 +481,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const float2 e = Erow[tt];
             yv[m] = (acc[m] + e.x) * e.y;
         }
-        if (!dvalid || nown <= 0) return;
+        if (chan_d(k) >= p.dim || nown <= 0) return;
         const int tmin = rv ? l0 + TT - 1 - (pos0 + R - 1) : l0 + pos0;
         float ya[R];                                      // time-ascending order
 #pragma unroll
@@ -506,51 +566,75 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll 1
         for (int blk = 0; blk < TT / 16; ++blk) {
             if (!FULL && blk * 16 >= nvalid) break;
-            float acc[16];
+            float acc[KC][16];
             if (FULL) {
-                // K steps at a time: their state-independent operands (shared-memory
-                // loads, delta*A, the SFU exps, delta*u*B) are all prepared first, as K
-                // independent streams, then the K dependent state updates run.
-                constexpr int K = SSM_SCAN_BATCH;
+                // KB steps at a time: their state-independent operands (shared-memory
+                // loads, delta*A, the SFU exps, delta*u*B) are all prepared first, then the
+                // KB dependent state updates run.
+                // (two channels per lane already give two independent update streams)
+                constexpr int KB = KC == 2 ? 1 : SSM_SCAN_BATCH;
 #pragma unroll
-                for (int q0 = 0; q0 < 16; q0 += K) {
-                    typename LaneState<NP, SUMMARY>::In in[K];
+                for (int q0 = 0; q0 < 16; q0 += KB) {
+                    typename LaneState<NP, SUMMARY>::In in[KB][KC];
 #pragma unroll
-                    for (int u = 0; u < K; ++u) {
+                    for (int u = 0; u < KB; ++u) {
                         const int tt = RV ? TT - 1 - (blk * 16 + q0 + u) : blk * 16 + q0 + u;
-                        in[u] = ls.prep(Prow[tt], Bl + tt * NS, Cl + tt * NS);
+                        float2 pd[KC];
+                        float bv[NP], cv[NP];
+                        load_p(tt, pd);
+                        load_bc(tt, bv, cv);
+#pragma unroll
+                        for (int k = 0; k < KC; ++k) in[u][k] = ls[k].prep(pd[k].x, pd[k].y, bv, cv);
                     }
 #pragma unroll
-                    for (int u = 0; u < K; ++u) acc[q0 + u] = ls.update(in[u]);
+                    for (int u = 0; u < KB; ++u)
+#pragma unroll
+                        for (int k = 0; k < KC; ++k) acc[k][q0 + u] = ls[k].update(in[u][k]);
                 }
             } else {
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const int ii = blk * 16 + q;
                     const int tt = RV ? TT - 1 - ii : ii;
-                    acc[q] = 0.f;
-                    if (ii < nvalid) acc[q] = ls.update(ls.prep(Prow[tt], Bl + tt * NS, Cl + tt * NS));
+#pragma unroll
+                    for (int k = 0; k < KC; ++k) acc[k][q] = 0.f;
+                    if (ii < nvalid) {
+                        float2 pd[KC];
+                        float bv[NP], cv[NP];
+                        load_p(tt, pd);
+                        load_bc(tt, bv, cv);
+#pragma unroll
+                        for (int k = 0; k < KC; ++k)
+                            acc[k][q] = ls[k].update(ls[k].prep(pd[k].x, pd[k].y, bv, cv));
+                    }
                 }
             }
             if (SUMMARY) continue;
-            reduce_block(acc);
             const int pos0 = blk * 16 + j * R;
-            epilogue(acc, RV, dir, l0, pos0, FULL ? R : max(0, min(R, nvalid - pos0)));
+#pragma unroll
+            for (int k = 0; k < KC; ++k) {
+                reduce_block(acc[k]);
+                epilogue(k, acc[k], RV, dir, l0, pos0, FULL ? R : max(0, min(R, nvalid - pos0)));
+            }
         }
     };
 
     auto finish_direction = [&](int dir) {
-        if (!dvalid) return;
-        if (SUMMARY) {
-            float2* sm = p.summary + (int64_t)chunk * p.batch * p.dim * NS + row * NS + j * NP;
 #pragma unroll
-            for (int k = 0; k < NP; ++k) sm[k] = make_float2(ls.get_pr(k), ls.get(k));
-        } else if (chunk == p.nchunks - 1 && p.final_state[dir]) {
-            float* fs = p.final_state[dir] + row * p.dstate;
+        for (int k = 0; k < KC; ++k) {
+            if (chan_d(k) >= p.dim) continue;
+            const int64_t row = chan_row(k);
+            if (SUMMARY) {
+                float2* sm = p.summary + (int64_t)chunk * p.batch * p.dim * NS + row * NS + j * NP;
 #pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const int n = j * NP + k;
-                if (n < p.dstate) fs[n] = ls.get(k);
+                for (int i = 0; i < NP; ++i) sm[i] = make_float2(ls[k].get_pr(i), ls[k].get(i));
+            } else if (chunk == p.nchunks - 1 && p.final_state[dir]) {
+                float* fs = p.final_state[dir] + row * p.dstate;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    const int n = j * NP + i;
+                    if (n < p.dstate) fs[n] = ls[k].get(i);
+                }
             }
         }
     };
@@ -572,7 +656,8 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             __syncthreads();                 // params of direction 0 no longer read
             load_params(1);
             load_A(1);
-            ls.reset();
+#pragma unroll
+            for (int k = 0; k < KC; ++k) ls[k].reset();
             __syncthreads();
         }
         bool ok = true;

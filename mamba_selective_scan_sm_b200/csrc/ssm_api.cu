@@ -123,20 +123,25 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
 
     const int es = elem_size(a->dtype);
     const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
-    int np = 4, s = 4;
+    int np = 4, s = 4, kc = 1;
     if (ns == 16) {
-        // 8 lanes per channel doubles the warps when batch*dim alone leaves the SMs short
+        // 8 lanes per channel doubles the warps when batch*dim alone leaves the SMs short.
+        // Two channels per lane (B and C registers shared) halve the shared-memory traffic
+        // of B and C per update but also the warp count; measured slower on B200 for the
+        // workloads here, so it is opt-in.
         const int64_t warps4 = a->batch * a->dim * 4 / 32;
         s = env_int("SSM_LANES_PER_CHANNEL", warps4 >= 2 * 4 * 148 ? 4 : 8);
         if (s != 4 && s != 8) s = 4;
         np = 16 / s;
+        kc = env_int("SSM_CHANNELS_PER_LANE", 1);
+        if (kc != 1 && kc != 2) kc = 1;
     } else if (ns == 8) {
         np = 2;
     } else {
         np = 1;
     }
-    if (!ssm::scan_variant(es, np, s, &pl->v))
-        return fail(SSM_ERR_UNSUPPORTED, "no kernel for elem %d np %d s %d", es, np, s);
+    if (!ssm::scan_variant(es, np, s, kc, &pl->v))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for elem %d np %d s %d kc %d", es, np, s, kc);
     pl->mode = bidir ? 2 : (a->reverse ? 1 : 0);
 
     const int tile = pl->v.tile;

@@ -105,7 +105,9 @@ def test_bidirectional_matches_oracle(dtype, conv, shape):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("reverse", [False, True])
 @pytest.mark.parametrize("chunks", [2, 3, 7, 100])
-def test_two_pass_chunk_carry(dtype, reverse, chunks):
+@pytest.mark.parametrize("per_lane", ["1", "2"])
+def test_two_pass_chunk_carry(monkeypatch, dtype, reverse, chunks, per_lane):
+    monkeypatch.setenv("SSM_CHANNELS_PER_LANE", per_lane)
     inp = synth.scan_inputs(1, 40, 1000, 16, dtype, conv_width=4, seed=14)
     y, h = _run(inp, dtype, reverse=reverse, conv=True, chunks=chunks)
     yo, ho = _oracle(inp, reverse=reverse, conv=True)
@@ -121,10 +123,12 @@ def test_two_pass_chunk_carry(dtype, reverse, chunks):
 
 
 @pytest.mark.parametrize("lanes", ["4", "8"])
+@pytest.mark.parametrize("per_lane", ["1", "2"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_lane_split_variants(monkeypatch, lanes, dtype):
-    """Both channel splits (4 or 8 lanes per channel) reach the same result."""
+def test_lane_split_variants(monkeypatch, lanes, per_lane, dtype):
+    """Every work split (4 or 8 lanes per channel, 1 or 2 channels per lane) matches."""
     monkeypatch.setenv("SSM_LANES_PER_CHANNEL", lanes)
+    monkeypatch.setenv("SSM_CHANNELS_PER_LANE", per_lane)
     inp = synth.scan_inputs(2, 40, 300, 16, dtype, conv_width=4, seed=15)
     for reverse in (False, True):
         y, h = _run(inp, dtype, reverse=reverse, conv=True)
