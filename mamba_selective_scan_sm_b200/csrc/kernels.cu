@@ -9,16 +9,16 @@ namespace ssm {
 
 namespace {
 
-template <typename T, int NP, int S, int KC>
+template <typename T, int NP, int S, int KC, int SW>
 ScanVariant variant_of() {
-    using Cfg = ScanCfg<T, NP, S, KC>;
-    return ScanVariant{(int)sizeof(T), NP, S, KC, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM};
+    using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    return ScanVariant{(int)sizeof(T), NP, S, KC, SW, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM};
 }
 
-template <typename T, int NP, int S, int KC, bool TMA, bool SUM>
+template <typename T, int NP, int S, int KC, int SW, bool TMA, bool SUM>
 cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
-    using Cfg = ScanCfg<T, NP, S, KC>;
-    auto* k = scan_fwd_kernel<T, NP, S, KC, TMA, SUM>;
+    using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    auto* k = scan_fwd_kernel<T, NP, S, KC, SW, TMA, SUM>;
     static const cudaError_t attr =
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (attr != cudaSuccess) return attr;
@@ -26,31 +26,33 @@ cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cud
     return cudaGetLastError();
 }
 
-template <typename T, int NP, int S, int KC>
+template <typename T, int NP, int S, int KC, int SW>
 cudaError_t launch_t(bool tma, bool sum, const ScanMaps& maps, const ScanParams& p, dim3 grid,
                      cudaStream_t st) {
-    if (tma) return sum ? launch_one<T, NP, S, KC, true, true>(maps, p, grid, st)
-                        : launch_one<T, NP, S, KC, true, false>(maps, p, grid, st);
-    return sum ? launch_one<T, NP, S, KC, false, true>(maps, p, grid, st)
-               : launch_one<T, NP, S, KC, false, false>(maps, p, grid, st);
+    if (tma) return sum ? launch_one<T, NP, S, KC, SW, true, true>(maps, p, grid, st)
+                        : launch_one<T, NP, S, KC, SW, true, false>(maps, p, grid, st);
+    return sum ? launch_one<T, NP, S, KC, SW, false, true>(maps, p, grid, st)
+               : launch_one<T, NP, S, KC, SW, false, false>(maps, p, grid, st);
 }
 
 }  // namespace
 
-// (states per lane, lanes per channel, channels per lane)
+// (states per lane, lanes per channel, channels per lane, scan warps per CTA)
+#ifndef SSM_SCAN_VARIANTS
 #define SSM_SCAN_VARIANTS(X) \
-    X(4, 4, 1)               \
-    X(4, 4, 2)               \
-    X(2, 8, 1)               \
-    X(2, 8, 2)               \
-    X(2, 4, 1)               \
-    X(1, 4, 1)
+    X(4, 4, 1, 4)            \
+    X(4, 4, 2, 2)            \
+    X(2, 8, 1, 2)            \
+    X(2, 8, 2, 4)            \
+    X(2, 4, 1, 4)            \
+    X(1, 4, 1, 4)
+#endif
 
-bool scan_variant(int es, int np, int s, int kc, ScanVariant* v) {
-#define X(NP_, S_, KC_)                                                     \
-    if (np == NP_ && s == S_ && kc == KC_) {                                \
-        *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_, KC_>()            \
-                     : variant_of<float, NP_, S_, KC_>();                   \
+bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
+#define X(NP_, S_, KC_, SW_)                                                \
+    if (np == NP_ && s == S_ && kc == KC_ && sw == SW_) {                   \
+        *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_, KC_, SW_>()       \
+                     : variant_of<float, NP_, S_, KC_, SW_>();              \
         return es == 2 || es == 4;                                          \
     }
     SSM_SCAN_VARIANTS(X)
@@ -60,11 +62,11 @@ bool scan_variant(int es, int np, int s, int kc, ScanVariant* v) {
 
 cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
                         const ScanParams& p, dim3 grid, cudaStream_t st) {
-#define X(NP_, S_, KC_)                                                                   \
-    if (v.np == NP_ && v.s == S_ && v.kc == KC_)                                          \
+#define X(NP_, S_, KC_, SW_)                                                              \
+    if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                           \
         return v.elem_size == 2                                                           \
-                   ? launch_t<__nv_bfloat16, NP_, S_, KC_>(tma, sum, maps, p, grid, st)   \
-                   : launch_t<float, NP_, S_, KC_>(tma, sum, maps, p, grid, st);
+                   ? launch_t<__nv_bfloat16, NP_, S_, KC_, SW_>(tma, sum, maps, p, grid, st) \
+                   : launch_t<float, NP_, S_, KC_, SW_>(tma, sum, maps, p, grid, st);
     SSM_SCAN_VARIANTS(X)
 #undef X
     return cudaErrorInvalidValue;

@@ -13,6 +13,7 @@ struct ScanVariant {
     int np;             // states per lane
     int s;              // lanes per channel
     int kc;             // channels per lane
+    int sw;             // scan warps per CTA
     int channels;       // channels per CTA
     int threads;        // threads per CTA
     int tile;           // time steps per tile (128 bytes of elements)
@@ -20,8 +21,8 @@ struct ScanVariant {
     int smem_bytes;     // dynamic shared memory per CTA
 };
 
-// Returns false if (elem_size, np, s, kc) has no compiled kernel.
-bool scan_variant(int elem_size, int np, int s, int kc, ScanVariant* v);
+// Returns false if (elem_size, np, s, kc, sw) has no compiled kernel.
+bool scan_variant(int elem_size, int np, int s, int kc, int sw, ScanVariant* v);
 
 cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, const ScanMaps& maps,
                         const ScanParams& p, dim3 grid, cudaStream_t stream);

@@ -1,22 +1,29 @@
 // Selective-scan forward kernel for sm_100a.
 //
-// Work split. A CTA of 128 threads owns G = 128/S channels of one batch row and
-// walks the sequence in tiles of TT = 32 time steps.
-// The S lanes of a channel each keep NP = NS/S of the (padded) NS states in
-// registers, so one channel's recurrence is spread over S lanes with no carry
-// between them (A is diagonal: the states never interact).
+// Work split. A CTA owns G channels of one batch row and walks the sequence in
+// tiles of TT steps (TT*sizeof(T) = 64 bytes). Its four warps have two roles:
 //
-// Per tile:
-//   1. TMA brings the raw tiles (u or the pre-conv x with a 16-byte halo, dt, z,
-//      B, C) into a 2-stage shared-memory ring; B and C are shared by the CTA's
-//      channels (all channels of a batch row read the same B_t, C_t).
-//   2. Prologue, once per (channel, t): conv + SiLU, delta = softplus(dt + bias),
-//      delta*u, D*u and silu(z) -> fp32 staging buffers; B and C are transposed to
-//      [t][n] fp32 so each lane reads its NP states with one vector load.
-//   3. Scan: per (t, state) one ex2 on the SFU, then h = dA*h + delta*u*B and the
-//      lane's partial C.h. Every 16 steps a butterfly transpose-reduce over the S
-//      lanes leaves each lane owning 16/S consecutive outputs, which it gates and
-//      stores with one vector store.
+//  * 2 producer warps own the TMA ring and the once-per-(channel, t) prologue. For
+//    each tile they wait for the raw tiles (u or the pre-conv x with a 16-byte halo,
+//    dt, z, B, C; B and C are shared by all channels of a batch row), compute
+//    conv + SiLU, delta = softplus(dt + bias), delta*u, D*u and silu(z) into one of
+//    two staging buffers, transpose B and C to fp32 [t][n], and hand the buffer
+//    over through an mbarrier;
+//  * 2 scan warps run the recurrence. The S lanes of a channel each keep NP = NS/S
+//    of the (padded) NS states in registers, so a channel's recurrence is spread
+//    over S lanes with no carry between them (A is diagonal: the states never
+//    interact); a lane serves KC channels with the same NP states, so each B and C
+//    value it reads from shared memory feeds KC updates. Per (t, state) one ex2 on
+//    the SFU, then h = dA*h + delta*u*B and the lane's partial C.h. Every 16 steps a
+//    butterfly transpose-reduce over the S lanes leaves each lane owning 16/S
+//    consecutive outputs of each of its channels, which it gates and stores with one
+//    vector store. The buffer goes back to the producers through a second mbarrier.
+//
+// The scan warps never stop at a CTA-wide barrier: the prologue of tile f + 1 runs
+// on the producer warps while the scan warps work through tile f. The scan is bound
+// by the SFU (one exp per state and step), the issue slots and the shared-memory
+// bandwidth together; serving KC channels per lane cuts the bytes each lane reads
+// per update.
 //
 // Two-pass chunk carry (paperlayer.ai summary of arXiv 2603.09555, §3 Method,
 // "Chunked recurrence"): with nchunks > 1, a SUMMARY launch scans every chunk but
@@ -36,20 +43,29 @@ namespace ssm {
 #define SSM_SCAN_BATCH 2
 #endif
 
+constexpr int kProWarps = 2;                                // TMA + prologue warps
+constexpr int kProThreads = 32 * kProWarps;                 // 64
+constexpr int kProBarrier = 1;                              // the producers' named barrier
+
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <typename T, int NP, int S, int KC>
+template <typename T, int NP, int S, int KC, int SW>
 struct ScanCfg {
-    static constexpr int G = S == 4 ? 32 : 16;          // channels per CTA
-    static constexpr int NT = G * S / KC;               // threads per CTA
-    static constexpr int NS = NP * S;         // padded state count
+    static constexpr int SCAN_THREADS = 32 * SW; // SW recurrence warps
+    static constexpr int G = SCAN_THREADS / S * KC;   // channels per CTA
+    static constexpr int NT = SCAN_THREADS + kProThreads;   // threads per CTA
+    // CTAs per SM the launch bounds ask for: three of 6 warps (96 registers per
+    // thread), three of 4 warps with two channels per lane (168), five of 4 warps (96)
+    static constexpr int MIN_CTAS = SW == 4 ? 3 : (KC == 2 ? 3 : 5);
+    static constexpr int NS = NP * S;            // padded state count
     static constexpr int ES = sizeof(T);
-    static constexpr int TT = 32;             // tile length (time steps)
-    static constexpr int ROWB = TT * ES;      // bytes of one tile row: 64 (bf16) / 128 (fp32)
-    static constexpr int SWZ = ROWB == 128 ? 7 : 3;   // TMA 128-B / 64-B swizzle mask
-    static constexpr int HALO = 16 / ES;      // conv history, one 16-B TMA granule
-    static constexpr int NSTAGE = 2;
-    static constexpr int R = 16 / S;          // outputs owned per lane per 16-step block
+    static constexpr int TT = 64 / ES;           // tile length: 32 (bf16) / 16 (fp32) steps
+    static constexpr int ROWB = TT * ES;         // bytes of one tile row (64)
+    static constexpr int SWZ = 3;                // TMA 64-B swizzle mask
+    static constexpr int HALO = 16 / ES;         // conv history, one 16-B TMA granule
+    static constexpr int NSTAGE = 2;             // raw TMA stages
+    static constexpr int NBUF = 2;               // staging buffers
+    static constexpr int R = 16 / S;             // outputs owned per lane, channel and block
     // raw stage (bytes from the 1024-aligned stage base)
     static constexpr int RAW_B = 0;                                   // [NS][TT], swizzled
     static constexpr int RAW_C = align_up(NS * ROWB, 1024);           // [NS][TT], swizzled
@@ -58,34 +74,53 @@ struct ScanCfg {
     static constexpr int RAW_DT = align_up(RAW_X + G * X_PITCH_MAX, 128);
     static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, 128);
     static constexpr int STAGE = align_up(RAW_Z + G * ROWB, 1024);
-    // fp32 staging. P: per channel group of KC channels and step, KC x {delta, delta*u}.
+    // Staging buffer (fp32). P: per group of KC channels and step, KC x {delta,
+    // delta*u} (one vector load per lane and step). E: per channel and step {D*u,
+    // silu(z)}. B and C transposed to [t][n], so a lane reads its NP states of a
+    // step with one vector load and no conversion.
     static constexpr int P_PITCH = TT * KC * 8 + 16;
-    static constexpr int E_PITCH = TT * 8 + 16;           // per channel: {D*u, silu(z)}
-    static constexpr int OFF_P = NSTAGE * STAGE;
-    static constexpr int OFF_E = OFF_P + (G / KC) * P_PITCH;
-    // Transposed B, C: [t][n] in the input type (bf16 stays bf16: exact, and half the
-    // shared-memory bytes each lane reads per step; fp32 stays fp32).
-    static constexpr int BCS = ES;
-    static constexpr int OFF_BT = align_up(OFF_E + G * E_PITCH, 16);
-    static constexpr int OFF_CT = OFF_BT + TT * NS * BCS;
-    static constexpr int OFF_PAR = align_up(OFF_CT + TT * NS * BCS, 16);  // 16 floats per channel
-    static constexpr int OFF_BAR = align_up(OFF_PAR + G * 64, 8);
-    static constexpr int BYTES = OFF_BAR + NSTAGE * 8;
-    static constexpr int SMEM = BYTES + 1024;             // slack for 1024-B alignment
+    static constexpr int E_PITCH = TT * 8 + 16;
+    static constexpr int BUF_P = 0;
+    static constexpr int BUF_E = (G / KC) * P_PITCH;
+    static constexpr int BUF_BT = BUF_E + G * E_PITCH;
+    static constexpr int BUF_CT = BUF_BT + TT * NS * 4;
+    static constexpr int BUF = align_up(BUF_CT + TT * NS * 4, 128);
+    static constexpr int OFF_BUF = NSTAGE * STAGE;
+    static constexpr int OFF_PAR = OFF_BUF + NBUF * BUF;   // [2 directions][G][16] floats
+    static constexpr int OFF_BAR = align_up(OFF_PAR + 2 * G * 64, 8);
+    static constexpr int NBARS = NSTAGE + 2 * NBUF;        // raw full; buffer full, empty
+    static constexpr int BYTES = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM = BYTES + 1024;              // slack for 1024-B alignment
     static_assert(TT % 16 == 0, "tile must hold whole 16-step blocks");
     static_assert(P_PITCH % 16 == 0 && E_PITCH % 16 == 0, "staging rows take 16-byte stores");
-    static_assert(G % 2 == 0, "the prologue pairs channel rows");
+    static_assert(BUF_E % 16 == 0 && BUF_BT % 16 == 0 && BUF % 16 == 0, "16-byte aligned parts");
     static_assert(NS <= 16, "at most 16 states");
     static_assert(KC == 1 || KC == 2, "one or two channels per lane");
 };
 
-// Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 128-B
-// and 64-B swizzles XOR address bits [4, 4+k) with bits [7, 7+k) (k = 3 or 2) of
-// the offset from a 1024-byte aligned tile base; SWZ is the k-bit mask.
+// Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 64-B
+// swizzle XORs address bits [4, 6) with bits [7, 9) of the offset from a 1024-byte
+// aligned tile base; SWZ is that 2-bit mask.
 template <int ROWB, int SWZ>
 __device__ __forceinline__ int swz(int row, int byte_in_row) {
     const int off = row * ROWB + byte_in_row;
     return off ^ (((off >> 7) & SWZ) << 4);
+}
+
+// Element i (a compile-time index once unrolled) of a run of 16-byte chunks of T,
+// widened to fp32 (a bf16 value is the high half of an fp32 bit pattern).
+template <typename T, int N>
+__device__ __forceinline__ float chunk_elem(const uint4 (&w)[N], int i) {
+    constexpr int EPC = 16 / (int)sizeof(T);
+    const uint4 c = w[i / EPC];
+    if constexpr (sizeof(T) == 2) {
+        const int k = (i % 8) / 2;
+        const uint32_t word = k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w;
+        return __uint_as_float((i & 1) ? (word & 0xffff0000u) : (word << 16));
+    } else {
+        const int k = i % 4;
+        return __uint_as_float(k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w);
+    }
 }
 
 // Recurrence state of one lane: NP states, held as fp32 pairs so the four
@@ -124,9 +159,9 @@ struct LaneState {
     }
 
     // Operands of one time step that do not depend on the state: the decay factors
-    // exp2(delta*a2), delta*u*B and C. Computing them one step ahead of the state
-    // update (software pipelining) overlaps the shared-memory loads and the SFU
-    // latency with the previous step's dependent FMAs.
+    // exp2(delta*a2), delta*u*B and C. Preparing several steps' operands before their
+    // updates overlaps the shared-memory loads and the SFU latency with the
+    // dependent FMAs.
     struct In {
         uint64_t dA[NPR > 0 ? NPR : 1], bu[NPR > 0 ? NPR : 1], cc[NPR > 0 ? NPR : 1];
         float dA1, bu1, c1;
@@ -171,13 +206,11 @@ struct LaneState {
     }
 };
 
-// Four CTAs per SM at least: 128 registers per thread with 128-thread CTAs, up to
-// 255 with the 64-thread CTAs of the two-channel variant (shared memory allows 5).
-template <typename T, int NP, int S, int KC, bool USE_TMA, bool SUMMARY>
-__global__ void __launch_bounds__(ScanCfg<T, NP, S, KC>::NT, 4)
+template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY>
+__global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
-    using Cfg = ScanCfg<T, NP, S, KC>;
-    constexpr int NT = Cfg::NT;
+    using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    constexpr int kScanWarps = SW, kScanThreads = Cfg::SCAN_THREADS, kCtaThreads = Cfg::NT;
     using E = Elem<T>;
     constexpr int G = Cfg::G, NS = Cfg::NS, TT = Cfg::TT, HALO = Cfg::HALO, R = Cfg::R;
     constexpr int ROWB = Cfg::ROWB, SWZ = Cfg::SWZ;
@@ -186,17 +219,14 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float2* Pbuf = reinterpret_cast<float2*>(smem + Cfg::OFF_P);
-    float2* Ebuf = reinterpret_cast<float2*>(smem + Cfg::OFF_E);
-    T* Bt = reinterpret_cast<T*>(smem + Cfg::OFF_BT);
-    T* Ct = reinterpret_cast<T*>(smem + Cfg::OFF_CT);
     float* par = reinterpret_cast<float*>(smem + Cfg::OFF_PAR);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full_raw = bars;                    // [NSTAGE] TMA bytes landed (1 arrival + tx)
+    uint64_t* full_buf = bars + NSTAGE;           // [NBUF] staging written (producer arrivals)
+    uint64_t* empty_buf = bars + NSTAGE + Cfg::NBUF;   // [NBUF] staging read (scan arrivals)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int lg = tid / S;         // lane group: channels lg*KC .. lg*KC + KC - 1 of the CTA
-    const int j = tid % S;          // state group of this lane
     const int b = blockIdx.y;
     const int d0 = blockIdx.x * G;
     const int L = p.seqlen;
@@ -209,97 +239,254 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     const bool has_z = !SUMMARY && p.z != nullptr;
     const bool conv = p.conv_w != nullptr;
     const int xpitch = conv ? Cfg::X_PITCH_MAX : TT * (int)sizeof(T);
-    auto chan_d = [&](int k) { return d0 + lg * KC + k; };             // channel k of the lane
-    auto chan_row = [&](int k) { return (int64_t)b * p.dim + chan_d(k); };  // its (b, d) row
+    using TrueT = std::integral_constant<bool, true>;
+    using FalseT = std::integral_constant<bool, false>;
 
     auto tile_rev = [&](int f) { return p.mode == 1 || (p.mode == 2 && f >= ntl); };
+    auto tile_dir = [&](int f) { return (p.mode == 2 && f >= ntl) ? 1 : 0; };
     // time of the first element of flat tile f
     auto tile_l0 = [&](int f) {
-        const int jt = f % ntl;
-        const int i0 = cs + jt * TT;
+        const int i0 = cs + (f % ntl) * TT;
         return tile_rev(f) ? L - i0 - TT : i0;
     };
+    auto buf_of = [&](int f) { return smem + Cfg::OFF_BUF + (f & 1) * Cfg::BUF; };
 
-    if (USE_TMA && tid == 0) {
-        for (int s = 0; s < NSTAGE; ++s) mbar_init(&bars[s], 1);
+    if (tid == 0) {
+        for (int s = 0; s < NSTAGE; ++s) mbar_init(&full_raw[s], 1);
+        for (int s = 0; s < Cfg::NBUF; ++s) {
+            mbar_init(&full_buf[s], kProThreads);
+            mbar_init(&empty_buf[s], kScanThreads);
+        }
         fence_mbar_init();
-        prefetch_tensormap(&maps.x);
-        prefetch_tensormap(&maps.dt);
-        prefetch_tensormap(&maps.B);
-        prefetch_tensormap(&maps.C);
-        if (has_z) prefetch_tensormap(&maps.z);
+    }
+    // Channel parameters of both directions -> smem, 16 floats per channel slot, each
+    // value twice so a 64-bit load yields the pair the packed prologue math needs:
+    // {w0,w0, w1,w1, w2,w2, w3,w3, conv_b x2, dt_bias x2, D x2, 0, 0}.
+    for (int e = tid; e < ndir * G; e += kCtaThreads) {
+        const int dir = e / G, r = e % G, dd = d0 + r;
+        float* q = par + (dir * G + r) * 16;
+        const bool ok = dd < p.dim;
+        // conv taps right-aligned: tap 3 meets the newest input
+        for (int k = 0; k < 4; ++k) {
+            const int kk = k - (4 - p.conv_width);
+            q[2 * k] = q[2 * k + 1] =
+                (ok && conv && kk >= 0) ? p.conv_w[(int64_t)dd * p.conv_width + kk] : 0.f;
+        }
+        q[8] = q[9] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
+        q[10] = q[11] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
+        q[12] = q[13] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
+        q[14] = q[15] = 0.f;
+    }
+    __syncthreads();   // barriers initialised and parameters written, for both roles
+
+    if (warp >= kScanWarps) {
+        // ============================================================ producers ==
+        const int ptid = tid - kScanThreads;
+
+        auto issue = [&](int f) {   // one thread: TMA loads of flat tile f
+            uint8_t* st = smem + (f % NSTAGE) * Cfg::STAGE;
+            const int l0 = tile_l0(f);
+            const bool rv = tile_rev(f);
+            const uint32_t bytes =
+                2u * NS * ROWB + G * xpitch + G * ROWB + (has_z ? G * ROWB : 0u);
+            uint64_t* bar = &full_raw[f % NSTAGE];
+            mbar_arrive_expect_tx(bar, bytes);
+            tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, l0, 0, b);
+            tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, l0, 0, b);
+            tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, (conv && !rv) ? l0 - HALO : l0, d0, b);
+            tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, l0, d0, b);
+            if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, l0, d0, b);
+        };
+
+        // Plain-load fallback (any alignment): fills stage 0 with the same layout.
+        auto load_plain = [&](int f) {
+            uint8_t* st = smem;
+            const int l0 = tile_l0(f);
+            const bool rv = tile_rev(f);
+            const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
+            const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
+            for (int e = ptid; e < NS * TT; e += kProThreads) {
+                const int n = e / TT, col = e % TT, t = l0 + col;
+                const bool ok = n < p.dstate && t >= 0 && t < L;
+                const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
+                *reinterpret_cast<T*>(st + Cfg::RAW_B + off) = ok ? gB[(int64_t)n * L + t] : T(0.f);
+                *reinterpret_cast<T*>(st + Cfg::RAW_C + off) = ok ? gC[(int64_t)n * L + t] : T(0.f);
+            }
+            const int xw = xpitch / (int)sizeof(T);
+            const int xs = (conv && !rv) ? l0 - HALO : l0;
+            for (int e = ptid; e < G * xw; e += kProThreads) {
+                const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
+                const bool ok = dd < p.dim && t >= 0 && t < L;
+                const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
+                reinterpret_cast<T*>(st + Cfg::RAW_X + r * xpitch)[col] =
+                    ok ? static_cast<const T*>(p.u)[gi] : T(0.f);
+            }
+            for (int e = ptid; e < G * TT; e += kProThreads) {
+                const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
+                const bool ok = dd < p.dim && t >= 0 && t < L;
+                const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
+                reinterpret_cast<T*>(st + Cfg::RAW_DT)[r * TT + col] =
+                    ok ? static_cast<const T*>(p.delta)[gi] : T(0.f);
+                if (has_z)
+                    reinterpret_cast<T*>(st + Cfg::RAW_Z)[r * TT + col] =
+                        ok ? static_cast<const T*>(p.z)[gi] : T(0.f);
+            }
+        };
+
+        // Raw stage `st` of tile f -> staging buffer `buf`. Each producer thread owns a
+        // segment of SEG consecutive steps of one channel row: it reads its window of x
+        // (with the conv history), dt and z with 16-byte loads, keeps the channel's
+        // parameters in registers, and works through SEG/2 independent step pairs.
+        auto prologue = [&](auto rv_tag, auto conv_tag, int f, const uint8_t* st, uint8_t* buf) {
+            constexpr bool RV = decltype(rv_tag)::value;
+            constexpr bool CONV = decltype(conv_tag)::value;
+            constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte chunk
+            // steps per producer thread (at least one chunk; then not every thread has one)
+            constexpr int SEG = TT * G / kProThreads > EPC ? TT * G / kProThreads : EPC;
+            constexpr int NSEG = TT * G / SEG;                // segments per tile
+            constexpr int SUB = 2 * EPC < SEG ? 2 * EPC : SEG;  // steps per register window
+            constexpr int NC = SUB / EPC;                     // dt / z chunks per window
+            constexpr int NXC = CONV ? NC + 1 : NC;           // x chunks (+ the conv history)
+            static_assert(SEG % SUB == 0 && SUB % EPC == 0 && SUB % 2 == 0, "windows of whole chunks");
+            // B, C: swizzled [n][t] -> fp32 [t][n], one 16-byte chunk per thread and pass
+            constexpr int NCH = NS * ROWB / 16;               // chunks per tensor
+            for (int e = ptid; e < 2 * NCH; e += kProThreads) {
+                const int ten = e / NCH, ch = e % NCH;
+                const int n = ch % NS, c0 = (ch / NS) * EPC;
+                const uint8_t* src =
+                    st + (ten ? Cfg::RAW_C : Cfg::RAW_B) + swz<ROWB, SWZ>(n, c0 * (int)sizeof(T));
+                const uint4 v[1] = {*reinterpret_cast<const uint4*>(src)};
+                float* dst = reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) + c0 * NS + n;
+#pragma unroll
+                for (int m = 0; m < EPC; ++m) dst[m * NS] = chunk_elem<T>(v, m);
+            }
+            if (NSEG < kProThreads && ptid >= NSEG) return;
+            const int r = ptid % G;                           // channel row
+            const int t0 = (ptid / G) * SEG;                  // first step of the segment
+            const uint4* q4 = reinterpret_cast<const uint4*>(par + (tile_dir(f) * G + r) * 16);
+            const uint4 qa = q4[0], qb = q4[1], qc = q4[2], qd = q4[3];
+            // duplicated pairs: {w0,w0} {w1,w1} {w2,w2} {w3,w3} {cb,cb} {bias,bias} {D,D}
+            const uint64_t w2[4] = {pk2(__uint_as_float(qa.x), __uint_as_float(qa.y)),
+                                    pk2(__uint_as_float(qa.z), __uint_as_float(qa.w)),
+                                    pk2(__uint_as_float(qb.x), __uint_as_float(qb.y)),
+                                    pk2(__uint_as_float(qb.z), __uint_as_float(qb.w))};
+            const uint64_t cb2 = pk2(__uint_as_float(qc.x), __uint_as_float(qc.y));
+            const uint64_t bias2 = pk2(__uint_as_float(qc.z), __uint_as_float(qc.w));
+            const uint64_t D2 = pk2(__uint_as_float(qd.x), __uint_as_float(qd.y));
+            // P rows hold KC channels side by side: this channel's {delta, delta*u} slot
+            uint8_t* prow_base = buf + Cfg::BUF_P + (r / KC) * Cfg::P_PITCH + (r % KC) * 8;
+#pragma unroll
+            for (int s0 = t0; s0 < t0 + SEG; s0 += SUB) {
+                // x window: row elements [s0, s0 + NXC*EPC). Forward rows start HALO steps
+                // before the tile (the conv history), reverse rows end HALO steps after it.
+                const uint4* xs = reinterpret_cast<const uint4*>(
+                    st + Cfg::RAW_X + r * (CONV ? Cfg::X_PITCH_MAX : ROWB) + s0 * (int)sizeof(T));
+                const uint4* ds =
+                    reinterpret_cast<const uint4*>(st + Cfg::RAW_DT + r * ROWB + s0 * (int)sizeof(T));
+                const uint4* zs =
+                    reinterpret_cast<const uint4*>(st + Cfg::RAW_Z + r * ROWB + s0 * (int)sizeof(T));
+                uint4 xw[NXC], dw[NC], zw[NC];
+#pragma unroll
+                for (int c2 = 0; c2 < NXC; ++c2) xw[c2] = xs[c2];
+#pragma unroll
+                for (int c2 = 0; c2 < NC; ++c2) {
+                    dw[c2] = ds[c2];
+                    zw[c2] = has_z ? zs[c2] : make_uint4(0, 0, 0, 0);
+                }
+                uint8_t* prow = prow_base + s0 * KC * 8;
+                uint8_t* erow = buf + Cfg::BUF_E + r * Cfg::E_PITCH + s0 * 8;
+#pragma unroll
+                for (int i = 0; i < SUB; i += 2) {           // steps s0 + i, s0 + i + 1
+                    uint64_t u2;
+                    if constexpr (CONV) {
+                        // forward: u_t = sum_k w_k x[t-3+k]; reverse: u_t = sum_k w_k x[t+3-k]
+                        uint64_t acc = cb2;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int a = RV ? i + 3 - k : HALO + i - 3 + k;
+                            acc = fma2(w2[k], pk2(chunk_elem<T>(xw, a), chunk_elem<T>(xw, a + 1)), acc);
+                        }
+                        u2 = silu2(acc);
+                    } else {
+                        u2 = pk2(chunk_elem<T>(xw, i), chunk_elem<T>(xw, i + 1));
+                    }
+                    uint64_t dl2 = add2(pk2(chunk_elem<T>(dw, i), chunk_elem<T>(dw, i + 1)), bias2);
+                    if (p.softplus) dl2 = softplus2(dl2);
+                    const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
+                    if constexpr (KC == 1) {
+                        *reinterpret_cast<float4*>(prow + i * 8) = make_float4(dl.x, du.x, dl.y, du.y);
+                    } else {
+                        *reinterpret_cast<float2*>(prow + i * KC * 8) = make_float2(dl.x, du.x);
+                        *reinterpret_cast<float2*>(prow + (i + 1) * KC * 8) = make_float2(dl.y, du.y);
+                    }
+                    if (!SUMMARY) {
+                        uint64_t g2 = pk2(1.f, 1.f);
+                        if (has_z) g2 = silu2(pk2(chunk_elem<T>(zw, i), chunk_elem<T>(zw, i + 1)));
+                        const float2 g = upk2(g2), dv = upk2(mul2(D2, u2));
+                        *reinterpret_cast<float4*>(erow + i * 8) = make_float4(dv.x, g.x, dv.y, g.y);
+                    }
+                }
+            }
+        };
+
+        if (USE_TMA && ptid == 0) {
+            prefetch_tensormap(&maps.x);
+            prefetch_tensormap(&maps.dt);
+            prefetch_tensormap(&maps.B);
+            prefetch_tensormap(&maps.C);
+            if (has_z) prefetch_tensormap(&maps.z);
+            for (int f = 0; f < min(NSTAGE, nt); ++f) issue(f);
+        }
+        for (int f = 0; f < nt; ++f) {
+            // Lane 0 of each warp polls (bounded); then every lane observes the completed
+            // phase itself with one try_wait, acquiring the writes it guards. A phase
+            // cannot move on before this warp's own part in the next round, so the
+            // parity test is unambiguous.
+            bool ok = true;
+            if (f >= Cfg::NBUF) {     // the scan warps are done with this buffer (tile f - 2)
+                const uint32_t par_e = ((f - Cfg::NBUF) / Cfg::NBUF) & 1;
+                if (lane == 0) ok = mbar_wait_bounded(&empty_buf[f & 1], par_e);
+                __syncwarp();
+                if (lane != 0) mbar_try_wait(&empty_buf[f & 1], par_e);
+            }
+            const uint8_t* st = smem;
+            if (USE_TMA) {
+                const uint32_t par_r = (f / NSTAGE) & 1;
+                if (lane == 0 && ok) ok = mbar_wait_bounded(&full_raw[f % NSTAGE], par_r);
+                __syncwarp();
+                if (lane != 0) mbar_try_wait(&full_raw[f % NSTAGE], par_r);
+                st = smem + (f % NSTAGE) * Cfg::STAGE;
+            } else {
+                // stage 0 was released by every producer at the end of tile f - 1
+                load_plain(f);
+            }
+            // one decision for all producers (this is also the barrier that orders the
+            // plain loads before the prologue): leave together if a wait ran out
+            if (named_bar_or(kProBarrier, kProThreads, !ok)) {
+                if (USE_TMA && ptid == 0)     // drain the copies still in flight (bounded)
+                    for (int g2 = f; g2 < min(f + NSTAGE, nt); ++g2)
+                        mbar_wait_bounded(&full_raw[g2 % NSTAGE], (g2 / NSTAGE) & 1);
+                return;
+            }
+            if (conv) {
+                if (tile_rev(f)) prologue(TrueT{}, TrueT{}, f, st, buf_of(f));
+                else prologue(FalseT{}, TrueT{}, f, st, buf_of(f));
+            } else {
+                if (tile_rev(f)) prologue(TrueT{}, FalseT{}, f, st, buf_of(f));
+                else prologue(FalseT{}, FalseT{}, f, st, buf_of(f));
+            }
+            mbar_arrive(&full_buf[f & 1]);
+            named_bar_sync(kProBarrier, kProThreads);   // every producer is done with the stage
+            if (USE_TMA && ptid == 0 && f + NSTAGE < nt) issue(f + NSTAGE);
+        }
+        return;
     }
 
-    auto issue = [&](int f) {   // one thread: TMA loads of flat tile f
-        uint8_t* st = smem + (f % NSTAGE) * Cfg::STAGE;
-        const int l0 = tile_l0(f);
-        const bool rv = tile_rev(f);
-        const uint32_t xbytes = G * xpitch;
-        uint32_t bytes = 2u * NS * ROWB + xbytes + G * ROWB + (has_z ? G * ROWB : 0u);
-        mbar_arrive_expect_tx(&bars[f % NSTAGE], bytes);
-        tma_load_3d(st + Cfg::RAW_B, &maps.B, &bars[f % NSTAGE], l0, 0, b);
-        tma_load_3d(st + Cfg::RAW_C, &maps.C, &bars[f % NSTAGE], l0, 0, b);
-        tma_load_3d(st + Cfg::RAW_X, &maps.x, &bars[f % NSTAGE], (conv && !rv) ? l0 - HALO : l0,
-                    d0, b);
-        tma_load_3d(st + Cfg::RAW_DT, &maps.dt, &bars[f % NSTAGE], l0, d0, b);
-        if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, &bars[f % NSTAGE], l0, d0, b);
-    };
-
-    // Plain-load fallback (any alignment): fills stage 0 with the same layout.
-    auto load_plain = [&](int f) {
-        uint8_t* st = smem;
-        const int l0 = tile_l0(f);
-        const bool rv = tile_rev(f);
-        const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
-        const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
-        for (int e = tid; e < NS * TT; e += NT) {
-            const int n = e / TT, col = e % TT, t = l0 + col;
-            const bool ok = n < p.dstate && t >= 0 && t < L;
-            const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
-            *reinterpret_cast<T*>(st + Cfg::RAW_B + off) = ok ? gB[(int64_t)n * L + t] : T(0.f);
-            *reinterpret_cast<T*>(st + Cfg::RAW_C + off) = ok ? gC[(int64_t)n * L + t] : T(0.f);
-        }
-        const int xw = xpitch / (int)sizeof(T);
-        const int xs = (conv && !rv) ? l0 - HALO : l0;
-        for (int e = tid; e < G * xw; e += NT) {
-            const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
-            const bool ok = dd < p.dim && t >= 0 && t < L;
-            const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
-            reinterpret_cast<T*>(st + Cfg::RAW_X + r * xpitch)[col] =
-                ok ? static_cast<const T*>(p.u)[gi] : T(0.f);
-        }
-        for (int e = tid; e < G * TT; e += NT) {
-            const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
-            const bool ok = dd < p.dim && t >= 0 && t < L;
-            const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
-            reinterpret_cast<T*>(st + Cfg::RAW_DT)[r * TT + col] =
-                ok ? static_cast<const T*>(p.delta)[gi] : T(0.f);
-            if (has_z)
-                reinterpret_cast<T*>(st + Cfg::RAW_Z)[r * TT + col] =
-                    ok ? static_cast<const T*>(p.z)[gi] : T(0.f);
-        }
-    };
-
-    // Per-direction channel parameters -> smem, 16 floats per channel slot, each value
-    // stored twice so a 64-bit load yields the pair the packed prologue math needs:
-    // {w0,w0, w1,w1, w2,w2, w3,w3, conv_b x2, dt_bias x2, D x2, 0, 0}.
-    auto load_params = [&](int dir) {
-        for (int e = tid; e < G; e += NT) {
-            const int dd = d0 + e;
-            float* q = par + e * 16;
-            const bool ok = dd < p.dim;
-            // conv taps right-aligned: tap 3 meets the newest input
-            for (int k = 0; k < 4; ++k) {
-                const int kk = k - (4 - p.conv_width);
-                q[2 * k] = q[2 * k + 1] =
-                    (ok && conv && kk >= 0) ? p.conv_w[(int64_t)dd * p.conv_width + kk] : 0.f;
-            }
-            q[8] = q[9] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
-            q[10] = q[11] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
-            q[12] = q[13] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
-            q[14] = q[15] = 0.f;
-        }
-    };
+    // =============================================================== scan warps ==
+    const int lg = tid / S;         // lane group: channels lg*KC .. lg*KC + KC - 1 of the CTA
+    const int j = tid % S;          // state group of this lane
+    auto chan_d = [&](int k) { return d0 + lg * KC + k; };                 // channel k of the lane
+    auto chan_row = [&](int k) { return (int64_t)b * p.dim + chan_d(k); };  // its (b, d) row
 
     LaneState<NP, SUMMARY> ls[KC];
     auto load_A = [&](int dir) {
@@ -339,140 +526,30 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    auto prologue = [&](int f, const uint8_t* st) {
-        const bool rv = tile_rev(f);
-        const int xoff = (conv && !rv) ? HALO : 0;
-        // B, C: swizzled [n][t] -> [t][n] in the input type, one 16-byte chunk per thread
-        constexpr int EPC = 16 / (int)sizeof(T);           // elements per 16-byte chunk
-        constexpr int NCH = NS * ROWB / 16;                // chunks per tensor
-        for (int e = tid; e < 2 * NCH; e += NT) {
-            const int ten = e / NCH, ch = e % NCH;
-            const int n = ch % NS, t0 = (ch / NS) * EPC;
-            const uint8_t* src = st + (ten ? Cfg::RAW_C : Cfg::RAW_B) + swz<ROWB, SWZ>(n, t0 * (int)sizeof(T));
-            T* dst = (ten ? Ct : Bt) + t0 * NS + n;
-            const uint4 v = *reinterpret_cast<const uint4*>(src);
-            const T* tv = reinterpret_cast<const T*>(&v);
+    // butterfly transpose-reduce over the S lanes of a channel: afterwards lane j
+    // holds the sums of block positions [j*R, j*R + R) in acc[0 .. R)
+    auto reduce_block = [&](float* acc) {
+        int len = 16;
 #pragma unroll
-            for (int m = 0; m < EPC; ++m) dst[m * NS] = tv[m];
-        }
-        // per (channel, t) quantities, two consecutive steps per lane in packed pairs:
-        // 16 lanes cover one 32-step channel row, a warp two rows at a time
-        for (int idx = warp; idx < G / 2; idx += NT / 32) {
-            const int r = 2 * idx + (lane >> 4);
-            const int tt = 2 * (lane & 15);                 // steps tt and tt + 1
-            const T* xr = reinterpret_cast<const T*>(st + Cfg::RAW_X + r * xpitch);
-            const uint64_t* q2 = reinterpret_cast<const uint64_t*>(par + r * 16);
-            uint64_t u2;
-            if (conv) {
-                // forward: u_t = sum_k w_k x[t-3+k]; reverse: u_t = sum_k w_k x[t+3-k]
-                float xv[5];
+        for (int m = S / 2; m >= 1; m >>= 1) {
+            const int half = len >> 1;
+            const bool upper = (j & m) != 0;
 #pragma unroll
-                for (int m = 0; m < 5; ++m)
-                    xv[m] = E::to_f(rv ? xr[tt + 4 - m] : xr[xoff + tt - 3 + m]);
-                uint64_t acc = q2[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    acc = fma2(q2[k], rv ? pk2(xv[k + 1], xv[k]) : pk2(xv[k], xv[k + 1]), acc);
-                u2 = silu2(acc);
-            } else {
-                u2 = pk2(E::to_f(xr[tt]), E::to_f(xr[tt + 1]));
+            for (int i = 0; i < half; ++i) {
+                const float send = upper ? acc[i] : acc[i + half];
+                const float keep = upper ? acc[i + half] : acc[i];
+                acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
             }
-            const T* dtr = reinterpret_cast<const T*>(st + Cfg::RAW_DT) + r * TT + tt;
-            uint64_t dl2 = add2(pk2(E::to_f(dtr[0]), E::to_f(dtr[1])), q2[5]);
-            if (p.softplus) dl2 = softplus2(dl2);
-            const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
-            uint8_t* prow = reinterpret_cast<uint8_t*>(Pbuf) + (r / KC) * Cfg::P_PITCH;
-            if (KC == 1) {
-                *reinterpret_cast<float4*>(prow + tt * 8) = make_float4(dl.x, du.x, dl.y, du.y);
-            } else {
-                *reinterpret_cast<float2*>(prow + tt * 16 + (r % KC) * 8) = make_float2(dl.x, du.x);
-                *reinterpret_cast<float2*>(prow + tt * 16 + 16 + (r % KC) * 8) = make_float2(dl.y, du.y);
-            }
-            if (!SUMMARY) {
-                uint64_t g2 = pk2(1.f, 1.f);
-                if (has_z) {
-                    const T* zr = reinterpret_cast<const T*>(st + Cfg::RAW_Z) + r * TT + tt;
-                    g2 = silu2(pk2(E::to_f(zr[0]), E::to_f(zr[1])));
-                }
-                const float2 g = upk2(g2), dv = upk2(mul2(q2[6], u2));
-                *reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(Ebuf) + r * Cfg::E_PITCH + tt * 8) =
-                    make_float4(dv.x, g.x, dv.y, g.y);
-            }
+            len = half;
         }
     };
 
-    const uint8_t* Prow = reinterpret_cast<uint8_t*>(Pbuf) + lg * Cfg::P_PITCH;
-    const T* Bl = Bt + j * NP;
-    const T* Cl = Ct + j * NP;
-    // P of step tt for the lane's KC channels: pd[k] = {delta, delta*u}
-    auto load_p = [&](int tt, float2 (&pd)[KC]) {
-        if constexpr (KC == 2) {
-            const float4 v = *reinterpret_cast<const float4*>(Prow + tt * 16);
-            pd[0] = make_float2(v.x, v.y);
-            pd[1] = make_float2(v.z, v.w);
-        } else {
-            pd[0] = *reinterpret_cast<const float2*>(Prow + tt * 8);
-        }
-    };
-    // this lane's NP values of B and C at step tt (bf16 pairs are widened in registers:
-    // the high half of a 32-bit word is already an fp32 bit pattern, the low half
-    // shifted up by 16 is one)
-    auto load_bc = [&](int tt, float (&bv)[NP], float (&cv)[NP]) {
-        if constexpr (sizeof(T) == 2 && NP % 2 == 0) {
-            uint32_t wb[NP / 2], wc[NP / 2];
-            if constexpr (NP == 4) {
-                const uint2 b2 = *reinterpret_cast<const uint2*>(Bl + tt * NS);
-                wb[0] = b2.x; wb[1] = b2.y;
-                if (!SUMMARY) {
-                    const uint2 c2 = *reinterpret_cast<const uint2*>(Cl + tt * NS);
-                    wc[0] = c2.x; wc[1] = c2.y;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < NP / 2; ++i) {
-                    wb[i] = reinterpret_cast<const uint32_t*>(Bl + tt * NS)[i];
-                    if (!SUMMARY) wc[i] = reinterpret_cast<const uint32_t*>(Cl + tt * NS)[i];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < NP / 2; ++i) {
-                bv[2 * i] = __uint_as_float(wb[i] << 16);
-                bv[2 * i + 1] = __uint_as_float(wb[i] & 0xffff0000u);
-                if (!SUMMARY) {
-                    cv[2 * i] = __uint_as_float(wc[i] << 16);
-                    cv[2 * i + 1] = __uint_as_float(wc[i] & 0xffff0000u);
-                }
-            }
-        } else if constexpr (sizeof(T) == 4 && NP % 4 == 0) {
-#pragma unroll
-            for (int i = 0; i < NP; i += 4) {
-                const float4 b4 = *reinterpret_cast<const float4*>(Bl + tt * NS + i);
-                bv[i] = b4.x; bv[i + 1] = b4.y; bv[i + 2] = b4.z; bv[i + 3] = b4.w;
-                if (!SUMMARY) {
-                    const float4 c4 = *reinterpret_cast<const float4*>(Cl + tt * NS + i);
-                    cv[i] = c4.x; cv[i + 1] = c4.y; cv[i + 2] = c4.z; cv[i + 3] = c4.w;
-                }
-            }
-        } else if constexpr (sizeof(T) == 4 && NP == 2) {
-            const float2 b2 = *reinterpret_cast<const float2*>(Bl + tt * NS);
-            bv[0] = b2.x; bv[1] = b2.y;
-            if (!SUMMARY) {
-                const float2 c2 = *reinterpret_cast<const float2*>(Cl + tt * NS);
-                cv[0] = c2.x; cv[1] = c2.y;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < NP; ++i) {
-                bv[i] = E::to_f(Bl[tt * NS + i]);
-                if (!SUMMARY) cv[i] = E::to_f(Cl[tt * NS + i]);
-            }
-        }
-    };
-    // gate, skip term, bidirectional partial and the store of R owned outputs
-    auto epilogue = [&](int k, const float* acc, bool rv, int dir, int l0, int pos0, int nown) {
-        const float2* Erow = reinterpret_cast<const float2*>(
-            reinterpret_cast<uint8_t*>(Ebuf) + (lg * KC + k) * Cfg::E_PITCH);
-        const int64_t row = chan_row(k);
+    // gate, skip term, bidirectional partial and the store of R owned outputs of the
+    // lane's channel k
+    auto epilogue = [&](const uint8_t* buf, int k, const float* acc, bool rv, int dir, int l0,
+                        int pos0, int nown) {
+        const float2* Erow =
+            reinterpret_cast<const float2*>(buf + Cfg::BUF_E + (lg * KC + k) * Cfg::E_PITCH);
         float yv[R];
 #pragma unroll
         for (int m = 0; m < R; ++m) {
@@ -489,7 +566,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         // valid ascending index range: forward [0, nown); reverse [R - nown, R)
         const int mlo = rv ? R - nown : 0;
         const int mhi = rv ? R : nown;
-        const int64_t gbase = row * L + tmin;
+        const int64_t gbase = chan_row(k) * L + tmin;
         if (p.mode == 2 && dir == 1) {
 #pragma unroll
             for (int m = 0; m < R; ++m)
@@ -536,43 +613,65 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    // butterfly transpose-reduce over the S lanes of a channel: afterwards lane j
-    // holds the sums of block positions [j*R, j*R + R) in acc[0 .. R)
-    auto reduce_block = [&](float* acc) {
-        int len = 16;
-#pragma unroll
-        for (int m = S / 2; m >= 1; m >>= 1) {
-            const int half = len >> 1;
-            const bool upper = (j & m) != 0;
-#pragma unroll
-            for (int i = 0; i < half; ++i) {
-                const float send = upper ? acc[i] : acc[i + half];
-                const float keep = upper ? acc[i + half] : acc[i];
-                acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-            }
-            len = half;
-        }
-    };
-
-    // One tile in scan order. RV: walk time downwards. FULL: all TT steps valid
-    // (no per-step predicate; shared-memory offsets are compile-time constants).
-    auto scan_tile = [&](auto rv_tag, auto full_tag, int f) {
+    // One tile in scan order from staging buffer `buf`. RV: walk time downwards.
+    // FULL: all TT steps valid (no per-step predicate; shared-memory offsets are
+    // compile-time constants).
+    auto scan_tile = [&](auto rv_tag, auto full_tag, int f, const uint8_t* buf) {
         constexpr bool RV = decltype(rv_tag)::value;
         constexpr bool FULL = decltype(full_tag)::value;
-        const int dir = (p.mode == 2 && f >= ntl) ? 1 : 0;
+        const int dir = tile_dir(f);
         const int i0 = cs + (f % ntl) * TT;
         const int nvalid = FULL ? TT : min(TT, ce - i0);
         const int l0 = RV ? L - i0 - TT : i0;
+        const uint8_t* Prow = buf + Cfg::BUF_P + lg * Cfg::P_PITCH;
+        const float* Bl = reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * NP;
+        const float* Cl = reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * NP;
+        // {delta, delta*u} of step tt for the lane's KC channels
+        auto load_p = [&](int tt, float2 (&pd)[KC]) {
+            if constexpr (KC == 2) {
+                const float4 v = *reinterpret_cast<const float4*>(Prow + tt * 16);
+                pd[0] = make_float2(v.x, v.y);
+                pd[1] = make_float2(v.z, v.w);
+            } else {
+                pd[0] = *reinterpret_cast<const float2*>(Prow + tt * 8);
+            }
+        };
+        // this lane's NP values of B and C at step tt
+        auto load_bc = [&](int tt, float (&bv)[NP], float (&cv)[NP]) {
+            if constexpr (NP % 4 == 0) {
+#pragma unroll
+                for (int i = 0; i < NP; i += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(Bl + tt * NS + i);
+                    bv[i] = b4.x; bv[i + 1] = b4.y; bv[i + 2] = b4.z; bv[i + 3] = b4.w;
+                    if (!SUMMARY) {
+                        const float4 c4 = *reinterpret_cast<const float4*>(Cl + tt * NS + i);
+                        cv[i] = c4.x; cv[i + 1] = c4.y; cv[i + 2] = c4.z; cv[i + 3] = c4.w;
+                    }
+                }
+            } else if constexpr (NP == 2) {
+                const float2 b2 = *reinterpret_cast<const float2*>(Bl + tt * NS);
+                bv[0] = b2.x; bv[1] = b2.y;
+                if (!SUMMARY) {
+                    const float2 c2 = *reinterpret_cast<const float2*>(Cl + tt * NS);
+                    cv[0] = c2.x; cv[1] = c2.y;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    bv[i] = Bl[tt * NS + i];
+                    if (!SUMMARY) cv[i] = Cl[tt * NS + i];
+                }
+            }
+        };
 #pragma unroll 1
         for (int blk = 0; blk < TT / 16; ++blk) {
             if (!FULL && blk * 16 >= nvalid) break;
             float acc[KC][16];
             if (FULL) {
                 // KB steps at a time: their state-independent operands (shared-memory
-                // loads, delta*A, the SFU exps, delta*u*B) are all prepared first, then the
-                // KB dependent state updates run.
-                // (two channels per lane already give two independent update streams)
-                constexpr int KB = KC == 2 ? 1 : SSM_SCAN_BATCH;
+                // loads, delta*A, the SFU exps, delta*u*B) are all prepared first, then
+                // the KB x KC independent state updates run.
+                constexpr int KB = SSM_SCAN_BATCH;
 #pragma unroll
                 for (int q0 = 0; q0 < 16; q0 += KB) {
                     typename LaneState<NP, SUMMARY>::In in[KB][KC];
@@ -614,7 +713,8 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll
             for (int k = 0; k < KC; ++k) {
                 reduce_block(acc[k]);
-                epilogue(k, acc[k], RV, dir, l0, pos0, FULL ? R : max(0, min(R, nvalid - pos0)));
+                epilogue(buf, k, acc[k], RV, dir, l0, pos0,
+                         FULL ? R : max(0, min(R, nvalid - pos0)));
             }
         }
     };
@@ -639,63 +739,34 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
 
-    // ------------------------------------------------------------- main loop --
-    load_params(0);
     load_A(0);
     init_state();
-    if (USE_TMA) {
-        __syncthreads();   // barrier init visible before any wait
-        if (tid == 0)
-            for (int f = 0; f < min(NSTAGE, nt); ++f) issue(f);
-    }
-    __syncthreads();
-
     for (int f = 0; f < nt; ++f) {
         if (p.mode == 2 && f == ntl) {       // second direction of the bidirectional sum
             finish_direction(0);
-            __syncthreads();                 // params of direction 0 no longer read
-            load_params(1);
             load_A(1);
 #pragma unroll
             for (int k = 0; k < KC; ++k) ls[k].reset();
-            __syncthreads();
         }
+        // wait for the staging buffer of tile f (same polling scheme as the producers);
+        // a warp whose wait ran out leaves, and the producers then run out of time on
+        // the buffer it never releases
+        const uint32_t par_f = (f / Cfg::NBUF) & 1;
         bool ok = true;
-        const uint8_t* st;
-        if (USE_TMA) {
-            // one lane per warp polls; __syncwarp hands the completed phase to the rest
-            if (lane == 0) ok = mbar_wait_bounded(&bars[f % NSTAGE], (f / NSTAGE) & 1);
-            __syncwarp();
-            // each lane then observes the completed phase itself (one try_wait, which
-            // succeeds at once), so the TMA writes are acquired by every reader
-            if (lane != 0) mbar_try_wait(&bars[f % NSTAGE], (f / NSTAGE) & 1);
-            st = smem + (f % NSTAGE) * Cfg::STAGE;
-        } else {
-            load_plain(f);
-            __syncthreads();
-            st = smem;
-        }
-        prologue(f, st);
-        if (__syncthreads_or(!ok)) {
-            // a tile never landed: drain what is still in flight (bounded), leave
-            if (USE_TMA && tid == 0)
-                for (int g2 = f; g2 < min(f + NSTAGE, nt); ++g2)
-                    mbar_wait_bounded(&bars[g2 % NSTAGE], (g2 / NSTAGE) & 1);
-            return;
-        }
-        if (USE_TMA && tid == 0 && f + NSTAGE < nt) issue(f + NSTAGE);
+        if (lane == 0) ok = mbar_wait_bounded(&full_buf[f & 1], par_f);
+        if (__any_sync(0xffffffffu, !ok)) return;
+        if (lane != 0) mbar_try_wait(&full_buf[f & 1], par_f);
+        const uint8_t* buf = buf_of(f);
         const bool rv = tile_rev(f);
         const bool full = cs + (f % ntl) * TT + TT <= ce;
-        using TrueT = std::integral_constant<bool, true>;
-        using FalseT = std::integral_constant<bool, false>;
         if (full) {
-            if (rv) scan_tile(TrueT{}, TrueT{}, f);
-            else scan_tile(FalseT{}, TrueT{}, f);
+            if (rv) scan_tile(TrueT{}, TrueT{}, f, buf);
+            else scan_tile(FalseT{}, TrueT{}, f, buf);
         } else {
-            if (rv) scan_tile(TrueT{}, FalseT{}, f);
-            else scan_tile(FalseT{}, FalseT{}, f);
+            if (rv) scan_tile(TrueT{}, FalseT{}, f, buf);
+            else scan_tile(FalseT{}, FalseT{}, f, buf);
         }
-        __syncthreads();
+        mbar_arrive(&empty_buf[f & 1]);      // the producers may refill it with tile f + 2
     }
     finish_direction(p.mode == 2 ? 1 : 0);
 }

@@ -123,25 +123,28 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
 
     const int es = elem_size(a->dtype);
     const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
-    int np = 4, s = 4, kc = 1;
+    int np = 4, s = 4, kc = 1, sw = 4;
     if (ns == 16) {
-        // 8 lanes per channel doubles the warps when batch*dim alone leaves the SMs short.
-        // Two channels per lane (B and C registers shared) halve the shared-memory traffic
-        // of B and C per update but also the warp count; measured slower on B200 for the
-        // workloads here, so it is opt-in.
-        const int64_t warps4 = a->batch * a->dim * 4 / 32;
-        s = env_int("SSM_LANES_PER_CHANNEL", warps4 >= 2 * 4 * 148 ? 4 : 8);
+        // Batch rows with enough channels for two 32-channel CTAs per SM: 4 lanes per
+        // channel (4 states each) in CTAs of 4 scan warps. Fewer channels: 8 lanes per
+        // channel in CTAs of 2 scan warps (8 channels each), for more CTAs and warps.
+        // SSM_LANES_PER_CHANNEL (4, 8) and SSM_CHANNELS_PER_LANE (1, 2) pick another
+        // compiled split.
+        const bool wide = a->batch * a->dim >= 2 * 148 * 32;
+        s = env_int("SSM_LANES_PER_CHANNEL", wide ? 4 : 8);
         if (s != 4 && s != 8) s = 4;
-        np = 16 / s;
         kc = env_int("SSM_CHANNELS_PER_LANE", 1);
         if (kc != 1 && kc != 2) kc = 1;
+        np = 16 / s;
+        sw = (s == 4) == (kc == 1) ? 4 : 2;
     } else if (ns == 8) {
         np = 2;
     } else {
         np = 1;
     }
-    if (!ssm::scan_variant(es, np, s, kc, &pl->v))
-        return fail(SSM_ERR_UNSUPPORTED, "no kernel for elem %d np %d s %d kc %d", es, np, s, kc);
+    if (!ssm::scan_variant(es, np, s, kc, sw, &pl->v))
+        return fail(SSM_ERR_UNSUPPORTED, "no kernel for elem %d np %d s %d kc %d sw %d", es, np, s,
+                    kc, sw);
     pl->mode = bidir ? 2 : (a->reverse ? 1 : 0);
 
     const int tile = pl->v.tile;
@@ -298,9 +301,10 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
         const auto& v = pl.v;
         const uint32_t xbox = a->conv_weight ? v.tile + v.halo : v.tile;
         const uint64_t L = a->seqlen, D = a->dim, Bn = a->batch, N = a->dstate;
-        // B, C tiles use the swizzle whose span equals one tile row (64 B bf16, 128 B fp32)
-        const CUtensorMapSwizzle bc =
-            v.tile * es == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+        // B, C tiles use the swizzle whose span equals one tile row (64 B: 32 bf16 or
+        // 16 fp32 steps)
+        if (v.tile * es != 64) return fail(SSM_ERR_UNSUPPORTED, "tile rows must be 64 bytes");
+        const CUtensorMapSwizzle bc = CU_TENSOR_MAP_SWIZZLE_64B;
         const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
         tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
               encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
