@@ -105,8 +105,8 @@ def kernel_source_digest() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(w):
-    """DRAM bytes (read + write) per launch of the workload's dominant kernel, from the
+def recorded_traffic(key):
+    """DRAM bytes (read + write) per launch of workload `key`'s dominant kernel, from the
     committed ncu summary, if that capture was taken of the current sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(path):
@@ -114,7 +114,7 @@ def recorded_traffic(w):
     digest = kernel_source_digest()
     for line in open(path):
         f = [x.strip() for x in line.strip().strip("|").split("|")]
-        if len(f) >= 3 and f[0] == w.name and f[2] == digest:
+        if len(f) >= 3 and f[0] == key and f[2] == digest:
             try:
                 return float(f[1])
             except ValueError:
@@ -464,7 +464,7 @@ def main():
                "frac": sfu_ach / sfu_peak, "exp2_per_launch": exps,
                "peak_kind": (f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
                              f"{sm_mhz:.0f} MHz (sampled SM clock)")}
-        traffic = recorded_traffic(w)
+        traffic = recorded_traffic(args.workload)
         if w.name.startswith("decode"):
             roof = dict(bound="hbm", **{k: hbm[k] for k in ("achieved", "peak", "unit", "frac")},
                         traffic=traffic, peak_kind=hbm["peak_kind"],
