@@ -101,6 +101,199 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
     }
 }
 
+// Streaming variant (dstate 16): a CTA owns kStreamRows consecutive channels, one per
+// thread, and walks a range of batch rows. Each thread keeps its channel's A (16
+// values), conv taps, dt bias and D in registers for the whole range; each batch
+// row's tile (the rows' fp32 state, conv state, x, dt, z, and the batch row's B_t and
+// C_t) streams through a kStreamStages-deep ring of 1-D bulk copies, so several
+// tiles are in flight per CTA while one is updated, and the updated state, conv
+// state and y leave with bulk stores. A thread updates its row's 16 states as packed
+// fp32 pairs; nothing is computed twice. One CTA barrier per tile. W is the conv
+// width (0: no conv). Requires dim % kStreamRows == 0, dstate == 16 and 16-byte
+// aligned bases (checked on the host).
+constexpr int kStreamRows = 128;
+constexpr int kStreamStages = 4;
+constexpr int kStreamThreads = kStreamRows;
+
+template <typename T, int W>
+struct StreamTile {
+    // byte offsets inside one stage (every part 16-byte aligned; bulk copies need it)
+    static constexpr int ES = sizeof(T);
+    static constexpr int STATE = 0;                                   // [rows][16] fp32
+    static constexpr int CONV = STATE + kStreamRows * 16 * 4;         // [rows][W] T
+    static constexpr int X = CONV + (kStreamRows * W * ES + 15) / 16 * 16;   // [rows] T
+    static constexpr int DT = X + kStreamRows * ES;
+    static constexpr int Z = DT + kStreamRows * ES;
+    static constexpr int Y = Z + kStreamRows * ES;                    // output
+    static constexpr int BT = Y + kStreamRows * ES;                   // [16] T
+    static constexpr int CT = BT + 16 * ES;
+    static constexpr int BYTES = (CT + 16 * ES + 127) / 128 * 128;
+    static_assert(X % 16 == 0 && DT % 16 == 0 && Z % 16 == 0 && Y % 16 == 0 && BT % 16 == 0 &&
+                  CT % 16 == 0, "bulk copies need 16-byte aligned parts");
+};
+
+// 4 values of T at an aligned shared address (8 or 16 bytes), widened to fp32
+template <typename T>
+__device__ __forceinline__ void load4(const uint8_t* src, float (&v)[4]) {
+    if constexpr (sizeof(T) == 2) {
+        const uint2 q = *reinterpret_cast<const uint2*>(src);
+        v[0] = __uint_as_float(q.x << 16); v[1] = __uint_as_float(q.x & 0xffff0000u);
+        v[2] = __uint_as_float(q.y << 16); v[3] = __uint_as_float(q.y & 0xffff0000u);
+    } else {
+        const float4 q = *reinterpret_cast<const float4*>(src);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    }
+}
+
+template <typename T, int W>
+__global__ void __launch_bounds__(kStreamThreads, 4) decode_stream_kernel(const DecodeParams p) {
+    using E = Elem<T>;
+    using Tl = StreamTile<T, W>;
+    constexpr bool CONV = W > 0;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ uint64_t full[kStreamStages];
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int dbase = blockIdx.x * kStreamRows;
+    const int d = dbase + tid;                        // this thread's channel
+    const int64_t nbatch = p.rows / p.dim;
+    const int per = (int)((nbatch + gridDim.y - 1) / gridDim.y);
+    const int64_t bfirst = (int64_t)blockIdx.y * per;
+    const int ntiles = (int)max((int64_t)0, min((int64_t)per, nbatch - bfirst));
+    if (ntiles == 0) return;                          // uniform over the CTA
+    const bool gate = p.z != nullptr;
+    const uint32_t cs_bytes = kStreamRows * W * sizeof(T);
+    const uint32_t v_bytes = kStreamRows * sizeof(T);
+    const uint32_t tile_bytes =
+        kStreamRows * 64 + cs_bytes + v_bytes * (gate ? 3 : 2) + 2 * 16 * sizeof(T);
+
+    auto stage = [&](int i) { return dsm + (i % kStreamStages) * Tl::BYTES; };
+    auto issue = [&](int i) {                         // one thread: the loads of tile i
+        uint8_t* s = stage(i);
+        const int64_t b = bfirst + i;
+        const int64_t r0 = b * p.dim + dbase;
+        uint64_t* bar = &full[i % kStreamStages];
+        mbar_arrive_expect_tx(bar, tile_bytes);
+        bulk_load(s + Tl::STATE, p.state + r0 * 16, kStreamRows * 64, bar);
+        if (CONV) bulk_load(s + Tl::CONV, static_cast<const T*>(p.conv_state) + r0 * W, cs_bytes, bar);
+        bulk_load(s + Tl::X, static_cast<const T*>(p.x) + r0, v_bytes, bar);
+        bulk_load(s + Tl::DT, static_cast<const T*>(p.dt) + r0, v_bytes, bar);
+        if (gate) bulk_load(s + Tl::Z, static_cast<const T*>(p.z) + r0, v_bytes, bar);
+        bulk_load(s + Tl::BT, static_cast<const T*>(p.Bt) + b * 16, 16 * sizeof(T), bar);
+        bulk_load(s + Tl::CT, static_cast<const T*>(p.Ct) + b * 16, 16 * sizeof(T), bar);
+    };
+
+    int issued = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kStreamStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+        for (; issued < min(kStreamStages, ntiles); ++issued) issue(issued);
+    }
+
+    // A thread walks its state row's four 16-byte chunks starting at chunk rot: the
+    // eight lanes of a quarter-warp then touch eight different bank groups although
+    // their rows are 64 bytes apart. A and B/C are read in the same rotated order.
+    const int rot = (lane >> 1) & 3;
+    // the channel's parameters, once for the whole range of batch rows
+    uint64_t a2[8];                                   // A * log2(e), as pairs, rotated
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 a4 =
+            __ldg(reinterpret_cast<const float4*>(p.A + (int64_t)d * 16) + ((q + rot) & 3));
+        a2[2 * q] = pk2(a4.x * kLog2e, a4.y * kLog2e);
+        a2[2 * q + 1] = pk2(a4.z * kLog2e, a4.w * kLog2e);
+    }
+    float w[W > 0 ? W : 1], cb = 0.f;
+    if constexpr (CONV) {
+#pragma unroll
+        for (int k = 0; k < W; ++k) w[k] = __ldg(p.conv_w + (int64_t)d * W + k);
+        cb = p.conv_b ? __ldg(p.conv_b + d) : 0.f;
+    }
+    const float dbias = p.dt_bias ? __ldg(p.dt_bias + d) : 0.f;
+    const float Dv = p.D ? __ldg(p.D + d) : 0.f;
+
+    // Tile i's data is complete when its barrier's phase (i / stages) & 1 completes.
+    // Lane 0 of each warp polls (bounded), the CTA barrier shares the verdict, and
+    // every thread then observes the phase itself (acquiring the copied bytes).
+    auto wait_tile = [&](int i) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(&full[i % kStreamStages], (i / kStreamStages) & 1);
+        return ok;
+    };
+    auto drain = [&](int from) {                      // thread 0, on the way out
+        if (tid != 0) return;
+        for (int g = from; g < issued; ++g)
+            mbar_wait_bounded(&full[g % kStreamStages], (g / kStreamStages) & 1);
+        bulk_wait_read();
+    };
+
+    __syncthreads();                                  // barrier init before any wait
+    if (__syncthreads_or(!wait_tile(0))) { drain(0); return; }
+    for (int i = 0; i < ntiles; ++i) {
+        uint8_t* s = stage(i);
+        mbar_try_wait(&full[i % kStreamStages], (i / kStreamStages) & 1);
+        const float xt = E::to_f(reinterpret_cast<const T*>(s + Tl::X)[tid]);
+        float xc = xt;
+        T* scv = reinterpret_cast<T*>(s + Tl::CONV) + tid * W;
+        T win[W > 0 ? W : 1];
+        if constexpr (CONV) {
+            // window after the shift: [conv_state[1 .. W-1], x_t]; w[W-1] meets x_t
+#pragma unroll
+            for (int k = 0; k < W; ++k) win[k] = scv[k];
+            float acc = fmaf(w[W - 1], xt, cb);
+#pragma unroll
+            for (int k = 0; k + 1 < W; ++k) acc = fmaf(w[k], E::to_f(win[k + 1]), acc);
+            xc = silu(acc);
+        }
+        float dl = E::to_f(reinterpret_cast<const T*>(s + Tl::DT)[tid]) + dbias;
+        if (p.softplus) dl = softplus(dl);
+        const uint64_t dd = pk2(dl, dl), uu = pk2(dl * xc, dl * xc);
+        float4* hp = reinterpret_cast<float4*>(s + Tl::STATE + tid * 64);
+        uint64_t acc2 = pk2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int ch = (q + rot) & 3;             // state chunk: states 4ch .. 4ch+3
+            float bv[4], cv[4];
+            load4<T>(s + Tl::BT + ch * 4 * sizeof(T), bv);
+            load4<T>(s + Tl::CT + ch * 4 * sizeof(T), cv);
+            const float4 h4 = hp[ch];
+            uint64_t h[2] = {pk2(h4.x, h4.y), pk2(h4.z, h4.w)};
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint64_t x = mul2(dd, a2[2 * q + k]);
+                const uint64_t dA = pk2(ex2(lo2(x)), ex2(hi2(x)));
+                h[k] = fma2(dA, h[k], mul2(uu, pk2(bv[2 * k], bv[2 * k + 1])));
+                acc2 = fma2(pk2(cv[2 * k], cv[2 * k + 1]), h[k], acc2);
+            }
+            hp[ch] = make_float4(lo2(h[0]), hi2(h[0]), lo2(h[1]), hi2(h[1]));
+        }
+        float y = lo2(acc2) + hi2(acc2) + Dv * xc;
+        if (gate) y *= silu(E::to_f(reinterpret_cast<const T*>(s + Tl::Z)[tid]));
+        reinterpret_cast<T*>(s + Tl::Y)[tid] = E::from_f(y);
+        if constexpr (CONV) {                         // shift the window, append x_t
+#pragma unroll
+            for (int k = 0; k + 1 < W; ++k) scv[k] = win[k + 1];
+            scv[W - 1] = reinterpret_cast<const T*>(s + Tl::X)[tid];
+        }
+        fence_proxy_async_smem();                     // generic writes -> bulk-store reads
+        const bool ok = i + 1 < ntiles ? wait_tile(i + 1) : true;
+        if (__syncthreads_or(!ok)) { drain(i + 1); return; }
+        if (tid == 0) {
+            const int64_t r0 = (bfirst + i) * p.dim + dbase;
+            bulk_store(p.state + r0 * 16, s + Tl::STATE, kStreamRows * 64);
+            if (CONV) bulk_store(static_cast<T*>(p.conv_state) + r0 * W, s + Tl::CONV, cs_bytes);
+            bulk_store(static_cast<T*>(p.out) + r0, s + Tl::Y, v_bytes);
+            bulk_commit();
+            // the stage of tile i - 1 is free once its stores have read it
+            if (i >= 1 && issued < ntiles) {
+                asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                issue(issued++);
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_read();
+}
+
 // Bulk-copy variant: one CTA updates kDecRows consecutive channels of one batch row.
 // Thread 0 moves the rows' state, conv state, x, dt and z into shared memory with
 // 1-D bulk async copies (a handful of instructions for ~10 KB in flight per CTA);

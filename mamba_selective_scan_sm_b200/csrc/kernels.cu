@@ -35,6 +35,17 @@ cudaError_t launch_t(bool tma, bool sum, const ScanMaps& maps, const ScanParams&
                : launch_one<T, NP, S, KC, SW, false, false>(maps, p, grid, st);
 }
 
+template <typename T, int W>
+cudaError_t launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+    constexpr int smem = kStreamStages * StreamTile<T, W>::BYTES;
+    auto* k = decode_stream_kernel<T, W>;
+    static const cudaError_t attr =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kStreamThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 // (states per lane, lanes per channel, channels per lane, scan warps per CTA)
@@ -90,6 +101,26 @@ cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) 
 }
 
 cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_t st) {
+    if (p.stream) {
+        // about four CTAs per SM, each a contiguous range of batch rows
+        const int64_t groups = p.dim / kStreamRows, batch = p.rows / p.dim;
+        int64_t split = (148 * 4 + groups - 1) / groups;
+        if (split > batch) split = batch;
+        if (split < 1) split = 1;
+        const dim3 grid((unsigned)groups, (unsigned)split);
+        const int W = p.conv_w ? p.conv_width : 0;
+#define SSM_STREAM_W(T_, W_) \
+        if (W == W_) return launch_stream<T_, W_>(p, grid, st);
+        if (es == 2) {
+            SSM_STREAM_W(__nv_bfloat16, 0) SSM_STREAM_W(__nv_bfloat16, 2)
+            SSM_STREAM_W(__nv_bfloat16, 3) SSM_STREAM_W(__nv_bfloat16, 4)
+        } else {
+            SSM_STREAM_W(float, 0) SSM_STREAM_W(float, 2) SSM_STREAM_W(float, 3)
+            SSM_STREAM_W(float, 4)
+        }
+#undef SSM_STREAM_W
+        return cudaErrorInvalidValue;
+    }
     if (p.bulk) {
         const dim3 grid((unsigned)(p.dim / kDecRows), (unsigned)(p.rows / p.dim));
         if (es == 2) decode_bulk_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);

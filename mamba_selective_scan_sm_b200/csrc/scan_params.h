@@ -68,6 +68,7 @@ struct DecodeParams {
     int dim, dstate, conv_width, softplus;
     int vec;            // dstate == 16 and state / A rows 16-byte aligned
     int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
+    int stream;         // streaming variant: dstate 16, dim % 128 == 0, 16-byte aligned bases
 };
 
 }  // namespace ssm

@@ -411,10 +411,21 @@ ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const vo
     p.conv_width = conv_weight ? conv_width : 0;
     p.softplus = dt_softplus ? 1 : 0;
     p.vec = dstate == 16 && aligned(state, 16) && aligned(A, 16);
-    // bulk-copy variant: 64-row groups of 16-byte aligned rows
-    p.bulk = dim % 64 == 0 && batch <= 65535 && aligned(state, 16) && aligned(x, 16) && aligned(dt, 16) &&
-             aligned(out, 16) && (!z || aligned(z, 16)) &&
-             (!conv_weight || aligned(conv_state, 16)) && env_int("SSM_DECODE_PLAIN", 0) == 0;
+    // Kernel choice. Streaming (the default where it applies): dstate 16, 128-channel
+    // groups, conv width 2..4 or none, 16-byte aligned bases for its bulk copies. Else the bulk-copy kernel
+    // (64-channel groups), else plain loads. SSM_DECODE_KERNEL = plain | bulk | stream
+    // restricts the choice (tests compare the kernels).
+    const bool base16 = aligned(state, 16) && aligned(x, 16) && aligned(dt, 16) &&
+                        aligned(out, 16) && (!z || aligned(z, 16)) &&
+                        (!conv_weight || aligned(conv_state, 16));
+    const char* want = getenv("SSM_DECODE_KERNEL");
+    const bool any = !want || !*want;
+    const bool plain = !any && strcmp(want, "plain") == 0;
+    p.stream = !plain && (any || strcmp(want, "stream") == 0) && dstate == 16 &&
+               dim % 128 == 0 && (!conv_weight || conv_width >= 2) && base16 &&
+               aligned(A, 16) && aligned(B_t, 16) && aligned(C_t, 16);
+    p.bulk = !plain && !p.stream && (any || strcmp(want, "bulk") == 0) && dim % 64 == 0 &&
+             batch <= 65535 && base16;
     cudaError_t e = ssm::launch_decode(es, (int)dstate, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return ok();

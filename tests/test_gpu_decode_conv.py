@@ -150,14 +150,17 @@ def test_decode_repeated_equals_scan_on_gpu(dtype):
     state_close(host(st), host(h), "state")
 
 
+@pytest.mark.parametrize("kernel", ["stream", "bulk"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dstate", [16, 5])
 @pytest.mark.parametrize("width", [4, 2, 3])
 @pytest.mark.parametrize("opts", [dict(), dict(conv=False), dict(gate=False, skip=False)],
                          ids=["full", "no-conv", "no-z-no-D"])
-def test_decode_bulk_path_matches_oracle(dtype, dstate, width, opts):
-    """Rows a multiple of 64 with 16-byte aligned bases take the bulk-copy kernel."""
-    B, D, steps = 2, 96, 6                       # 192 rows = 3 bulk groups
+def test_decode_fast_paths_match_oracle(monkeypatch, kernel, dtype, dstate, width, opts):
+    """Channel counts a multiple of 64 with 16-byte aligned bases take the streaming
+    kernel (dstate 16) or the bulk-copy kernel; other dstates fall back to plain loads."""
+    monkeypatch.setenv("SSM_DECODE_KERNEL", kernel)
+    B, D, steps = 2, 128, 6
     inp = synth.decode_inputs(B, D, dstate, steps, width, dtype, seed=27)
     yg, sg, cg = _decode_gpu(inp, dtype, steps, **opts)
     yo, so, co = _decode_oracle(inp, steps, **opts)
@@ -168,13 +171,32 @@ def test_decode_bulk_path_matches_oracle(dtype, dstate, width, opts):
         np.testing.assert_array_equal(cg, co)
 
 
-def test_decode_bulk_and_plain_paths_agree(monkeypatch):
-    B, D, steps = 2, 128, 4
-    inp = synth.decode_inputs(B, D, 16, steps, 4, "bf16", seed=28)
-    yb, sb, cb = _decode_gpu(inp, "bf16", steps)
-    monkeypatch.setenv("SSM_DECODE_PLAIN", "1")
-    yp, sp, cp = _decode_gpu(inp, "bf16", steps)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_stream_many_batch_rows_per_cta(dtype):
+    """Enough batch rows that each CTA of the streaming kernel walks more tiles than its
+    copy ring has stages (200 rows in ranges of 14), with a ragged last range."""
+    B, D, steps = 200, 5120, 2
+    inp = synth.decode_inputs(B, D, 16, steps, 4, dtype, seed=29)
+    yg, sg, cg = _decode_gpu(inp, dtype, steps)
+    yo, so, co = _decode_oracle(inp, steps)
     for s in range(steps):
-        assert_bf16_ulp(yb[s], yp[s], f"step {s}")
-    state_close(sb, sp, "state")
-    np.testing.assert_array_equal(cb, cp)
+        assert_close_out(yg[s], yo[s], dtype, f"y step {s}")
+    state_close(sg, so, "state")
+    np.testing.assert_array_equal(cg, co)
+
+
+def test_decode_kernels_agree(monkeypatch):
+    """Streaming, bulk-copy and plain-load kernels give the same steps."""
+    B, D, steps = 3, 256, 4
+    inp = synth.decode_inputs(B, D, 16, steps, 4, "bf16", seed=28)
+    res = {}
+    for kernel in ("stream", "bulk", "plain"):
+        monkeypatch.setenv("SSM_DECODE_KERNEL", kernel)
+        res[kernel] = _decode_gpu(inp, "bf16", steps)
+    yp, sp, cp = res["plain"]
+    for kernel in ("stream", "bulk"):
+        yk, sk, ck = res[kernel]
+        for s in range(steps):
+            assert_bf16_ulp(yk[s], yp[s], f"{kernel} step {s}")
+        state_close(sk, sp, f"{kernel} state")
+        np.testing.assert_array_equal(ck, cp)
