@@ -93,15 +93,20 @@ def exp_count(w) -> int:
 
 # ---------------------------------------------------------------- traffic --
 
-def kernel_source_digest() -> str:
-    """sha256 over the CUDA sources of the library (what an ncu capture describes)."""
+KERNEL_SOURCES = {
+    "scan": ("scan_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu"),
+    "decode": ("decode_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu"),
+}
+
+
+def kernel_source_digest(kind: str) -> str:
+    """sha256 over the CUDA sources of one kernel family (what an ncu capture describes)."""
     import hashlib
     d = os.path.join(ROOT, "mamba_selective_scan_sm_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
@@ -111,7 +116,7 @@ def recorded_traffic(key):
     path = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(path):
         return None
-    digest = kernel_source_digest()
+    digest = kernel_source_digest("decode" if key.startswith("decode") else "scan")
     for line in open(path):
         f = [x.strip() for x in line.strip().strip("|").split("|")]
         if len(f) >= 3 and f[0] == key and f[2] == digest:
