@@ -41,7 +41,7 @@ def load_library(path: str):
     L = ctypes.c_long
     I = ctypes.c_int
     lib.oracle_causal_conv1d.argtypes = [P, P, P, P, L, L, L, I, I]
-    lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, P, I, I, P, P, I, P, P, P,
+    lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, P, I, I, P, P, I, P, P, P, P,
                                           L, L, L, L]
     lib.oracle_state_update.argtypes = [P, P, P, P, P, P, P, P, P, P, I, P, P, I, P, L, L, L]
     for f in (lib.oracle_causal_conv1d, lib.oracle_selective_scan, lib.oracle_state_update):
@@ -78,14 +78,19 @@ def causal_conv1d(x, w, bias=None, apply_silu=True):
 
 
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
-                   reverse=False, conv_w=None, conv_b=None, h0=None, return_final_state=False):
+                   reverse=False, conv_w=None, conv_b=None, h0=None, return_final_state=False,
+                   conv_hist=None):
     """One-direction scan. u, delta, z (B, D, L); B, C (B, N, L); A (D, N).
 
     With ``conv_w`` (D, W) given, ``u`` is the pre-conv x and the scan input is
-    silu(conv(x) + conv_b). Returns y (B, D, L) [and the final state (B, D, N)].
+    silu(conv(x) + conv_b). ``h0`` (B, D, N) is the initial state; ``conv_hist``
+    (B, D, W-1) holds the inputs before position 0, oldest first (forward only).
+    Returns y (B, D, L) [and the final state (B, D, N)].
     """
     u, delta, A, B, C = _d(u), _d(delta), _d(A), _d(B), _d(C)
     D, z, delta_bias, conv_w, conv_b, h0 = _d(D), _d(z), _d(delta_bias), _d(conv_w), _d(conv_b), _d(h0)
+    conv_hist = _d(conv_hist)
+    assert conv_hist is None or (conv_w is not None and not reverse)
     Bsz, Dm, L = u.shape
     N = A.shape[1]
     assert delta.shape == u.shape and B.shape == (Bsz, N, L) and C.shape == (Bsz, N, L)
@@ -95,9 +100,19 @@ def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_sof
     W = conv_w.shape[1] if conv_w is not None else 0
     _load().oracle_selective_scan(_p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z),
                                   _p(delta_bias), int(bool(delta_softplus)), int(bool(reverse)),
-                                  _p(conv_w), _p(conv_b), W, _p(h0), _p(out), _p(fs),
-                                  Bsz, Dm, L, N)
+                                  _p(conv_w), _p(conv_b), W, _p(h0), _p(conv_hist), _p(out),
+                                  _p(fs), Bsz, Dm, L, N)
     return (out, fs) if return_final_state else out
+
+
+def conv_tail(x, W, conv_hist=None):
+    """The last W inputs of the sequence conv_hist ++ x (zeros before either), oldest
+    first: the conv state a decode step or a following scan continues from."""
+    x = _d(x)
+    Bsz, Dm, L = x.shape
+    hist = np.zeros((Bsz, Dm, W - 1)) if conv_hist is None else _d(conv_hist)
+    full = np.concatenate([np.zeros((Bsz, Dm, 1)), hist, x], axis=2)
+    return full[:, :, -W:].copy()
 
 
 def selective_scan_bidir(u, delta, A, B, C, D, z, delta_bias, A_rev, D_rev, delta_bias_rev,

@@ -36,6 +36,13 @@
  *  - the reverse final state is the state after position 0 (its last step).
  *  - decode conv state holds the last W inputs, newest last; it shifts left by one
  *    and appends x_t before the convolution.
+ *  - a forward scan may continue a sequence processed earlier (a prompt taken in
+ *    pieces, or a prefill after decode steps): it then starts from that sequence's
+ *    state h0 and its conv reads the W-1 inputs that preceded position 0 (conv_hist,
+ *    oldest first) where it would otherwise read zeros. The pages carry the conv and
+ *    SSM states across calls in the step method and the inference cache (pyshine.com
+ *    tour, the block paragraph; paperlayer.ai summary, §3 Method, "Autoregressive
+ *    cache"); the same two states let a scan pick up where another call stopped.
  *
  * Parity pins: every function here is checked, on CPU, against closed forms,
  * brute-force products and invariants that do not call it twice the same way.
@@ -75,13 +82,15 @@ void oracle_causal_conv1d(const double* x, const double* w, const double* bias, 
  * u, delta, z, out: (Bsz, D, L); Bm, Cm: (Bsz, N, L); A: (D, N);
  * Dv, delta_bias, conv_b: (D) or NULL; conv_w: (D, W) or NULL (NULL: no conv);
  * h0: (Bsz, D, N) initial state or NULL (zeros); final_state: (Bsz, D, N) or NULL.
+ * conv_hist: (Bsz, D, W-1) inputs at positions -(W-1) .. -1, oldest first, or NULL
+ * (zeros); forward scans only.
  * reverse = 0 walks t = 0..L-1, reverse = 1 walks t = L-1..0. */
 void oracle_selective_scan(const double* u, const double* delta, const double* A,
                            const double* Bm, const double* Cm, const double* Dv,
                            const double* z, const double* delta_bias, int delta_softplus,
                            int reverse, const double* conv_w, const double* conv_b,
-                           int conv_width, const double* h0, double* out,
-                           double* final_state, long Bsz, long D, long L, long N) {
+                           int conv_width, const double* h0, const double* conv_hist,
+                           double* out, double* final_state, long Bsz, long D, long L, long N) {
     double h[1024];
     if (N > 1024) return;
     for (long b = 0; b < Bsz; ++b)
@@ -102,7 +111,11 @@ void oracle_selective_scan(const double* u, const double* delta, const double* A
                     for (int k = 0; k < conv_width; ++k) {
                         /* forward: x[t-W+1+k]; reverse (flipped sequence): x[t+W-1-k] */
                         long s = reverse ? t + (conv_width - 1) - k : t - (conv_width - 1) + k;
-                        if (s >= 0 && s < L) acc += conv_w[d * conv_width + k] * ur[s];
+                        if (s >= 0 && s < L)
+                            acc += conv_w[d * conv_width + k] * ur[s];
+                        else if (s < 0 && !reverse && conv_hist)  /* s in [-(W-1), -1] */
+                            acc += conv_w[d * conv_width + k] *
+                                   conv_hist[(b * D + d) * (conv_width - 1) + (conv_width - 1) + s];
                     }
                     ut = silu(acc);
                 } else {

@@ -53,6 +53,10 @@ MUTANTS = [
     ("decode dt bias dropped", "double dl = dt[bd] + (dt_bias ? dt_bias[d] : 0.0);",
      "double dl = dt[bd];", None),
     ("decode skip term dropped", "if (Dv) y += Dv[d] * xc;", "", None),
+    ("conv history read in reverse order", "(conv_width - 1) + s]", "-1 - s]", None),
+    ("conv history ignored", "else if (s < 0 && !reverse && conv_hist)", "else if (0 && conv_hist)",
+     None),
+    ("initial state ignored", "h[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;", "h[n] = 0.0;", None),
 ]
 
 

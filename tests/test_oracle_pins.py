@@ -365,6 +365,89 @@ def test_two_pass_chunk_carry_matches_sequential():
     np.testing.assert_allclose(H, h, rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------ continuing a sequence ---
+
+def _scan(c, sl=lambda a: a, **kw):
+    return oracle.selective_scan(sl(c["u"]), sl(c["delta"]), c["A"], sl(c["B"]), sl(c["C"]),
+                                 c["D"], sl(c["z"]), c["delta_bias"], True, False,
+                                 c.get("conv_w"), c.get("conv_b"), return_final_state=True, **kw)
+
+
+@pytest.mark.parametrize("W", [2, 3, 4])
+def test_conv_history_is_the_conv_of_the_joined_sequence(W):
+    """The scan input with a conv history equals the plain causal conv (pinned against
+    torch above) of history ++ x: run the scan over the joined sequence with B = 0 on the
+    history positions (they then leave the zero state untouched) and drop their outputs."""
+    rng = np.random.default_rng(15)
+    c = _rand_case(rng, 2, 3, 19, 4, conv=W)
+    hist = rng.standard_normal((2, 3, W - 1))
+    y, h = _scan(c, conv_hist=hist)
+    j = dict(c)
+    pad = lambda a, v: np.concatenate([v, a], axis=-1)
+    j["u"] = pad(c["u"], hist)
+    for k in ("delta", "z", "C"):
+        j[k] = pad(c[k], rng.standard_normal(c[k].shape[:-1] + (W - 1,)))
+    j["B"] = pad(c["B"], np.zeros((2, 4, W - 1)))
+    yj, hj = _scan(j)
+    np.testing.assert_array_equal(y, yj[..., W - 1:])
+    np.testing.assert_array_equal(h, hj)
+    # torch's conv1d over the joined sequence gives the same scan input
+    xj = torch.from_numpy(j["u"])
+    ref = torch.nn.functional.conv1d(xj, torch.from_numpy(c["conv_w"])[:, None, :],
+                                     torch.from_numpy(c["conv_b"]), padding=W - 1,
+                                     groups=3)[..., W - 1:W - 1 + 19].numpy()
+    y_unfused, _ = oracle.selective_scan(_silu(ref), c["delta"], c["A"], c["B"], c["C"], c["D"],
+                                         c["z"], c["delta_bias"], True, False,
+                                         return_final_state=True)
+    np.testing.assert_allclose(y, y_unfused, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("cuts", [(1,), (2,), (3,), (5,), (20,), (36,), (2, 3), (1, 2, 30)])
+def test_split_sequence_continues_from_state_and_history(cuts):
+    """Scanning a sequence in pieces, each from the previous piece's final state and the
+    last W-1 inputs before it, reproduces the one-piece scan (pieces shorter than W-1
+    included, so the history spans pieces)."""
+    rng = np.random.default_rng(16)
+    W, L = 4, 37
+    c = _rand_case(rng, 2, 3, L, 5, conv=W)
+    y, h = _scan(c)
+    bounds = [0, *cuts, L]
+    ys, st, hist = [], None, None
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        sl = lambda v: v[..., a:b]
+        yp, st = _scan(c, sl, h0=st, conv_hist=hist)
+        hist = oracle.conv_tail(sl(c["u"]), W, hist)[..., 1:]
+        ys.append(yp)
+    np.testing.assert_allclose(np.concatenate(ys, axis=-1), y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(st, h, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_continues_a_scan():
+    """Decode steps from a scan's final state and conv tail reproduce the rest of the
+    one-piece scan."""
+    rng = np.random.default_rng(17)
+    W, L, k = 4, 25, 9
+    c = _rand_case(rng, 2, 3, L, 4, conv=W)
+    y, h = _scan(c)
+    _, st = _scan(c, lambda v: v[..., :k])
+    cs = oracle.conv_tail(c["u"][..., :k], W)
+    for t in range(k, L):
+        yt, st, cs = oracle.state_update(st, cs, c["u"][..., t], c["delta"][..., t], c["A"],
+                                         c["B"][..., t], c["C"][..., t], c["D"], c["z"][..., t],
+                                         c["delta_bias"], True, c["conv_w"], c["conv_b"])
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st, h, rtol=1e-12, atol=1e-13)
+
+
+def test_conv_tail_layout():
+    """conv_tail: the last W inputs of history ++ x, zeros before both, oldest first."""
+    x = np.arange(1, 6, dtype=np.float64).reshape(1, 1, 5)           # 1..5
+    np.testing.assert_array_equal(oracle.conv_tail(x, 4), [[[2, 3, 4, 5]]])
+    np.testing.assert_array_equal(oracle.conv_tail(x[..., :2], 4), [[[0, 0, 1, 2]]])
+    np.testing.assert_array_equal(oracle.conv_tail(x[..., :1], 4, np.array([[[7, 8, 9]]])),
+                                  [[[7, 8, 9, 1]]])
+
+
 def test_oracle_consumes_bf16_rounded_inputs():
     """The synthetic generator rounds to bf16 first; the rounding is nearest-even."""
     x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.0 ** -130, 3.0e38], dtype=np.float32)
