@@ -67,7 +67,7 @@ extern "C" {
 #define SSM_API
 #endif
 
-#define SSM_ABI_VERSION 1
+#define SSM_ABI_VERSION 2
 #define SSM_MAX_DSTATE 16
 #define SSM_MAX_CONV_WIDTH 4
 
@@ -140,6 +140,19 @@ typedef struct {
     size_t workspace_bytes;
     int32_t num_chunks;       /* 0 = automatic; 1 = single pass; k > 1 = two-pass carry over
                                  k chunks of the sequence (one direction only) */
+    /* Continuing a sequence that an earlier call (a scan or decode steps) stopped at;
+     * forward single-direction scans only (ABI 2). */
+    const float* initial_state; /* (batch, dim, dstate) fp32 state before position 0, or
+                                   NULL (zeros) */
+    const void* conv_history; /* (batch, dim, conv_width - 1) in dtype: the inputs at
+                                 positions -(conv_width-1) .. -1, oldest first, that the
+                                 fused conv reads instead of zeros; or NULL. Needs
+                                 conv_weight. */
+    void* conv_state_out;     /* (batch, dim, conv_width) in dtype, or NULL: the last
+                                 conv_width inputs of conv_history ++ u, oldest first
+                                 (zeros before both) -- the conv state a decode step or
+                                 the next scan continues from. Needs conv_weight; must not
+                                 overlap the inputs. */
 } ssm_scan_args_t;
 
 /* Bytes of device workspace the call with these arguments needs (0 if none).
@@ -148,7 +161,17 @@ SSM_API ssm_status_t ssm_selective_scan_workspace_size(const ssm_scan_args_t* ar
 
 /* Selective-scan forward. See the file comment for the computation and the
  * struct fields for layouts. final_state is the state after the last step of the
- * scan direction (position seqlen-1 forward, position 0 reverse). */
+ * scan direction (position seqlen-1 forward, position 0 reverse).
+ * Continuation (forward, one direction): with initial_state and conv_history the
+ * scan picks up a sequence where an earlier call stopped, so a prompt can be taken
+ * in pieces and a prefill can follow decode steps or precede them; final_state and
+ * conv_state_out are what the next call (a scan, or ssm_selective_state_update)
+ * continues from. The pages carry these two states across calls for the step method
+ * (pyshine.com tour, block paragraph; paperlayer.ai §3 Method, "Autoregressive
+ * cache"). Errors: SSM_ERR_UNSUPPORTED for any of initial_state, conv_history,
+ * conv_state_out with reverse or the bidirectional sum; SSM_ERR_NULL_ARG for
+ * conv_history or conv_state_out without conv_weight; SSM_ERR_ALIAS when
+ * conv_state_out overlaps u, conv_history or out. */
 SSM_API ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* args, ssm_stream_t stream);
 
 /*

@@ -101,14 +101,18 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                            delta_softplus=True, reverse=False, conv_weight=None, conv_bias=None,
                            A_rev=None, D_rev=None, delta_bias_rev=None, *, out=None,
                            return_final_state=False, final_state=None, final_state_rev=None,
-                           num_chunks=0, workspace=None, stream=None):
+                           num_chunks=0, workspace=None, stream=None, initial_state=None,
+                           conv_history=None, conv_state_out=None, return_conv_state=False):
     """Selective-scan forward (see include/ssm.h). Layouts: u, delta, z (batch, dim, seqlen);
     B, C (batch, dstate, seqlen); A (dim, dstate) fp32. With ``conv_weight`` (dim, width), ``u``
     is the pre-conv x. With ``A_rev`` the result is the bidirectional sum.
 
     ``final_state`` / ``final_state_rev`` may be given as preallocated fp32 outputs
-    (batch, dim, dstate); they are written whenever given.
-    Returns ``out`` or ``(out, final_state[, final_state_rev])``.
+    (batch, dim, dstate); they are written whenever given. A forward scan continues a
+    sequence from ``initial_state`` (batch, dim, dstate) fp32 and ``conv_history``
+    (batch, dim, width - 1); ``conv_state_out`` (batch, dim, width), allocated when
+    ``return_conv_state``, receives the conv state the next call continues from.
+    Returns ``out``, or a tuple ``(out[, final_state[, final_state_rev]][, conv_state])``.
     """
     torch = _torch()
     lib = _abi.load()
@@ -121,8 +125,15 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
             fs = torch.empty(shp, dtype=torch.float32, device=u.device)
         if A_rev is not None and fsr is None:
             fsr = torch.empty(shp, dtype=torch.float32, device=u.device)
+    cs = conv_state_out
+    if return_conv_state and cs is None:
+        cs = torch.empty(u.shape[0], u.shape[1], conv_weight.shape[1], dtype=u.dtype,
+                         device=u.device)
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
                    conv_bias, A_rev, D_rev, delta_bias_rev, out, fs, fsr, num_chunks)
+    a.initial_state = _fp32(initial_state, "initial_state")
+    a.conv_history = _ptr(conv_history)
+    a.conv_state_out = _ptr(cs)
     n = ctypes.c_size_t()
     _abi.check(lib, lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     if n.value:
@@ -130,9 +141,12 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
             workspace = torch.empty(n.value, dtype=torch.uint8, device=u.device)
         a.workspace, a.workspace_bytes = _ptr(workspace), n.value
     _abi.check(lib, lib.ssm_selective_scan_fwd(ctypes.byref(a), _stream(stream)))
-    if not return_final_state:
-        return out
-    return (out, fs, fsr) if A_rev is not None else (out, fs)
+    res = [out]
+    if return_final_state:
+        res += [fs, fsr] if A_rev is not None else [fs]
+    if return_conv_state:
+        res.append(cs)
+    return res[0] if len(res) == 1 else tuple(res)
 
 
 def ssm_causal_conv1d_fwd(x, w, bias=None, apply_silu=True, *, out=None, stream=None):

@@ -22,6 +22,7 @@ EXPORTS = (
     "ssm_device_error", "ssm_selective_scan_fwd_noalloc",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
+ABI_VERSION = 2            # SSM_ABI_VERSION of include/ssm.h this mirror follows
 
 _P = ctypes.c_void_p
 _FP = ctypes.POINTER(ctypes.c_float)
@@ -41,6 +42,7 @@ class ScanArgs(ctypes.Structure):
         ("out", _P), ("final_state", _P), ("final_state_rev", _P),
         ("workspace", _P), ("workspace_bytes", ctypes.c_size_t),
         ("num_chunks", _I32),
+        ("initial_state", _P), ("conv_history", _P), ("conv_state_out", _P),
     ]
 
 
@@ -82,6 +84,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _P]
     lib.ssm_device_error.restype = ctypes.c_int
     lib.ssm_device_error.argtypes = [ctypes.POINTER(_I32), _P]
+    if lib.ssm_abi_version() != ABI_VERSION:
+        raise LibraryMissing(f"{path} implements ABI {lib.ssm_abi_version()}, this binding "
+                             f"expects {ABI_VERSION}: rebuild the library")
     if path == LIB_PATH:
         _lib = lib
     return lib

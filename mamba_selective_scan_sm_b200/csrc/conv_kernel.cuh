@@ -86,4 +86,21 @@ __global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
     }
 }
 
+// The conv state a scan leaves for the next call: per row, the last `width` inputs
+// of history ++ x, oldest first, zeros before both (one thread per row; a few
+// bytes per row).
+template <typename T>
+__global__ void __launch_bounds__(256) conv_tail_kernel(const ConvTailParams p) {
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= p.rows) return;
+    const int W = p.width, L = p.seqlen;
+    const T* x = static_cast<const T*>(p.x) + row * L;
+    const T* h = p.hist ? static_cast<const T*>(p.hist) + row * (W - 1) : nullptr;
+    T* o = static_cast<T*>(p.out) + row * W;
+    for (int k = 0; k < W; ++k) {
+        const int t = L - W + k;                       // position in the sequence
+        o[k] = t >= 0 ? x[t] : (h && t >= -(W - 1) ? h[W - 1 + t] : T(0.f));
+    }
+}
+
 }  // namespace ssm

@@ -83,6 +83,14 @@ cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps
     return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_conv_tail(int es, const ConvTailParams& p, cudaStream_t st) {
+    const int64_t blocks = (p.rows + 255) / 256;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (es == 2) conv_tail_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p);
+    else conv_tail_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) {
     const int64_t per_row = (p.seqlen + 7) / 8;
     const unsigned bx = (unsigned)((per_row + 127) / 128);

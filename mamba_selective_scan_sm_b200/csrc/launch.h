@@ -29,6 +29,8 @@ cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, const 
 
 cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream_t stream);
 
+cudaError_t launch_conv_tail(int elem_size, const ConvTailParams& p, cudaStream_t stream);
+
 cudaError_t launch_decode(int elem_size, int dstate, const DecodeParams& p, cudaStream_t stream);
 
 // Replace the calling thread's ssm_last_error_detail() text.

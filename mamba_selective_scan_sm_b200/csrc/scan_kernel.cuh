@@ -206,6 +206,22 @@ struct LaneState {
     }
 };
 
+// Writes the caller's conv history (the inputs at positions -(W-1) .. -1) into the
+// first forward tile's halo in shared memory. Out of line: it runs once per CTA and
+// keeps its registers out of the producer loop.
+template <typename T, int G, int HALO, int NTHR>
+__device__ __noinline__ void put_conv_history(const ScanParams& p, uint8_t* raw_x, int xpitch,
+                                              int ptid, int b, int d0) {
+    const int hw = p.conv_width - 1;
+    for (int e = ptid; e < G * hw; e += NTHR) {
+        const int r = e / hw, k = e % hw, dd = d0 + r;
+        if (dd < p.dim)
+            reinterpret_cast<T*>(raw_x + r * xpitch)[HALO - hw + k] =
+                static_cast<const T*>(p.conv_hist)[((int64_t)b * p.dim + dd) * hw + k];
+    }
+    fence_proxy_async_smem();                     // before the stage's next TMA write
+}
+
 template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY>
 __global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
@@ -314,12 +330,17 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             }
             const int xw = xpitch / (int)sizeof(T);
             const int xs = (conv && !rv) ? l0 - HALO : l0;
+            const int hw = conv ? p.conv_width - 1 : 0;      // history length
             for (int e = ptid; e < G * xw; e += kProThreads) {
                 const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
+                // positions before 0 read the caller's conv history, if any
+                const bool hist = p.conv_hist && !rv && dd < p.dim && t < 0 && t >= -hw;
+                const int64_t hi = ((int64_t)b * p.dim + dd) * hw + hw + t;
                 reinterpret_cast<T*>(st + Cfg::RAW_X + r * xpitch)[col] =
-                    ok ? static_cast<const T*>(p.u)[gi] : T(0.f);
+                    ok ? static_cast<const T*>(p.u)[gi]
+                       : (hist ? static_cast<const T*>(p.conv_hist)[hi] : T(0.f));
             }
             for (int e = ptid; e < G * TT; e += kProThreads) {
                 const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
@@ -456,6 +477,11 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 __syncwarp();
                 if (lane != 0) mbar_try_wait(&full_raw[f % NSTAGE], par_r);
                 st = smem + (f % NSTAGE) * Cfg::STAGE;
+                // The first forward tile's conv halo (positions < 0) landed as zeros;
+                // a continued sequence puts the caller's history there.
+                if (conv && p.conv_hist && p.mode == 0 && chunk == 0 && f == 0)
+                    put_conv_history<T, G, HALO, kProThreads>(p, smem + Cfg::RAW_X, xpitch, ptid,
+                                                               b, d0);
             } else {
                 // stage 0 was released by every producer at the end of tile f - 1
                 load_plain(f);
@@ -504,14 +530,18 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         }
     };
     // Initial state of this chunk: carry over the summaries of earlier chunks.
+    // A caller's initial state (a continued sequence) is the carry into chunk 0.
     auto init_state = [&]() {
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             ls[k].reset();
-            if (!SUMMARY && chunk > 0 && chan_d(k) < p.dim) {
+            if (!SUMMARY && (chunk > 0 || p.h0) && chan_d(k) < p.dim) {
                 float hv[NP];
 #pragma unroll
-                for (int i = 0; i < NP; ++i) hv[i] = 0.f;
+                for (int i = 0; i < NP; ++i) {
+                    const int n = j * NP + i;
+                    hv[i] = (p.h0 && n < p.dstate) ? p.h0[chan_row(k) * p.dstate + n] : 0.f;
+                }
                 const int64_t stride = (int64_t)p.batch * p.dim * NS;
                 for (int k2 = 0; k2 < chunk; ++k2) {
                     const float2* sm = p.summary + k2 * stride + chan_row(k) * NS + j * NP;

@@ -36,7 +36,19 @@ struct ScanParams {
     int chunk_len;          // scan positions per chunk (multiple of the tile length)
     int nchunks;
     float2* summary;        // two-pass: [nchunks-1][batch*dim][NS] {prod dA, h_end}
+    const float* h0;        // (batch, dim, dstate) state before position 0, or nullptr
+    const void* conv_hist;  // (batch, dim, conv_width-1) inputs before position 0, or nullptr
     int vec_store;          // rows are 16-byte aligned: vector stores allowed
+};
+
+// The last conv_width inputs of history ++ x per row (the conv state a decode step
+// continues from).
+struct ConvTailParams {
+    const void* x;          // (rows, seqlen)
+    const void* hist;       // (rows, width-1) or nullptr
+    void* out;              // (rows, width)
+    int64_t rows;
+    int seqlen, width;
 };
 
 // Standalone causal conv1d.

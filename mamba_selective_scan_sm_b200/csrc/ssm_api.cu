@@ -120,6 +120,12 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         return fail(SSM_ERR_UNSUPPORTED, "final_state_rev needs A_rev (bidirectional)");
     if (bidir && a->num_chunks > 1)
         return fail(SSM_ERR_UNSUPPORTED, "the bidirectional sum runs as a single pass");
+    const bool cont = a->initial_state || a->conv_history || a->conv_state_out;
+    if (cont && (bidir || a->reverse))
+        return fail(SSM_ERR_UNSUPPORTED,
+                    "initial_state, conv_history and conv_state_out need a forward scan");
+    if ((a->conv_history || a->conv_state_out) && !a->conv_weight)
+        return fail(SSM_ERR_NULL_ARG, "conv_history / conv_state_out need conv_weight");
 
     const int es = elem_size(a->dtype);
     const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
@@ -228,7 +234,9 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
         {a->conv_weight, 4, "conv_weight"}, {a->conv_bias, 4, "conv_bias"},
         {a->A_rev, 4, "A_rev"}, {a->D_rev, 4, "D_rev"}, {a->delta_bias_rev, 4, "delta_bias_rev"},
         {a->final_state, 4, "final_state"}, {a->final_state_rev, 4, "final_state_rev"},
-        {a->workspace, 16, "workspace"}};
+        {a->workspace, 16, "workspace"}, {a->initial_state, 4, "initial_state"},
+        {a->conv_history, (size_t)es, "conv_history"},
+        {a->conv_state_out, (size_t)es, "conv_state_out"}};
     for (auto& x : al)
         if (x.p && !aligned(x.p, x.al))
             return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", x.n, x.al);
@@ -238,18 +246,45 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
             overlap(a->out, act, a->C, bc))
             return fail(SSM_ERR_ALIAS, "out overlaps an input");
     }
+    const size_t st_bytes = (size_t)rows * a->dstate * sizeof(float);
+    const int cw = a->conv_weight ? a->conv_width : 0;
+    const size_t hist_bytes = cw > 0 ? (size_t)rows * (cw - 1) * es : 0;
+    const size_t tail_bytes = (size_t)rows * cw * es;
+    if (a->conv_state_out &&
+        (overlap(a->conv_state_out, tail_bytes, a->u, act) ||
+         overlap(a->conv_state_out, tail_bytes, a->conv_history, hist_bytes) ||
+         overlap(a->conv_state_out, tail_bytes, a->out, act)))
+        return fail(SSM_ERR_ALIAS, "conv_state_out overlaps u, conv_history or out");
+    // one pass reads a row's initial state before writing its final state; the two-pass
+    // carry reads it in every chunk while the last chunk writes the final state
+    if (pl.nchunks > 1 && overlap(a->final_state, st_bytes, a->initial_state, st_bytes))
+        return fail(SSM_ERR_ALIAS, "final_state overlaps initial_state with a two-pass carry");
     if (pl.workspace > 0 && (!a->workspace || a->workspace_bytes < pl.workspace))
         return fail(SSM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", pl.workspace,
                     a->workspace ? a->workspace_bytes : (size_t)0);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the conv state the next call continues from (independent of the scan's results)
+    auto conv_tail = [&]() -> ssm_status_t {
+        if (!a->conv_state_out || rows == 0) return SSM_OK;
+        ssm::ConvTailParams tp{a->u, a->conv_history, a->conv_state_out, rows, (int)a->seqlen, cw};
+        cudaError_t e = ssm::launch_conv_tail(es, tp, s);
+        return e == cudaSuccess ? SSM_OK : cuda_fail(e, "conv state launch");
+    };
     if (empty) {
-        // zero steps: the final state is the (zero) initial state
+        // zero steps: the final state is the initial state, the conv state its history
         const size_t fs = (size_t)rows * a->dstate * sizeof(float);
-        if (fs && a->final_state) {
+        if (fs && a->final_state && a->initial_state) {
+            if (a->final_state != a->initial_state) {
+                cudaError_t e = cudaMemcpyAsync(a->final_state, a->initial_state, fs,
+                                                cudaMemcpyDeviceToDevice, s);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
+            }
+        } else if (fs && a->final_state) {
             cudaError_t e = cudaMemsetAsync(a->final_state, 0, fs, s);
             if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
         }
+        if (ssm_status_t t = conv_tail(); t != SSM_OK) return t;
         if (fs && a->final_state_rev) {
             cudaError_t e = cudaMemsetAsync(a->final_state_rev, 0, fs, s);
             if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
@@ -285,6 +320,8 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     p.nchunks = pl.nchunks;
     uint8_t* ws = static_cast<uint8_t*>(a->workspace);
     p.summary = pl.summary_bytes ? reinterpret_cast<float2*>(ws) : nullptr;
+    p.h0 = a->initial_state;
+    p.conv_hist = a->conv_weight ? a->conv_history : nullptr;
     if (bidir)
         p.partial = a->dtype == SSM_F32
                         ? static_cast<float*>(a->out)
@@ -322,6 +359,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     }
     e = ssm::launch_scan(pl.v, tma, false, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    if (ssm_status_t t = conv_tail(); t != SSM_OK) return t;
     return ok();
 }
 

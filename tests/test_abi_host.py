@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.ssm_abi_version() == 1
+    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 2
     for code, name in _abi.STATUS.items():
         assert lib.ssm_status_string(code)
     assert lib.ssm_status_string(999) == b"unknown status"
@@ -93,6 +93,47 @@ def test_scan_conv_width_and_bidirectional_chunks(lib):
     assert _scan(lib, _args(conv_weight=FAKE + (1 << 30), conv_width=5)) == 2
     a = _args(A_rev=FAKE + (1 << 30), num_chunks=4)
     assert _scan(lib, a) == _abi.STATUS_CODE["SSM_ERR_UNSUPPORTED"]
+
+
+CONV = dict(conv_weight=FAKE + (1 << 30), conv_width=4)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(initial_state=FAKE + (1 << 29), reverse=1), "SSM_ERR_UNSUPPORTED"),
+    (dict(initial_state=FAKE + (1 << 29), A_rev=FAKE + (1 << 30)), "SSM_ERR_UNSUPPORTED"),
+    (dict(conv_history=FAKE + (1 << 29), reverse=1, **CONV), "SSM_ERR_UNSUPPORTED"),
+    (dict(conv_history=FAKE + (1 << 29)), "SSM_ERR_NULL_ARG"),
+    (dict(conv_state_out=FAKE + (1 << 29)), "SSM_ERR_NULL_ARG"),
+    (dict(initial_state=FAKE + (1 << 29) + 2), "SSM_ERR_MISALIGNED"),
+    (dict(conv_history=FAKE + (1 << 29) + 1, **CONV), "SSM_ERR_MISALIGNED"),
+    (dict(conv_state_out=FAKE + 64, **CONV), "SSM_ERR_ALIAS"),                 # inside u
+    (dict(conv_state_out=FAKE + 5 * (1 << 24) + 64, **CONV), "SSM_ERR_ALIAS"),  # inside out
+    (dict(conv_state_out=FAKE + (1 << 29), conv_history=FAKE + (1 << 29) + 96, **CONV),
+     "SSM_ERR_ALIAS"),
+    (dict(initial_state=FAKE + (1 << 29), final_state=FAKE + (1 << 29) + 64, num_chunks=4,
+          seqlen=4096, workspace=FAKE + (1 << 31), workspace_bytes=1 << 20), "SSM_ERR_ALIAS"),
+])
+def test_scan_continuation_arguments(lib, kw, status):
+    """initial_state / conv_history / conv_state_out: forward scans, a fused conv for the
+    conv ones, aligned, and outputs that do not overlap what the scan reads."""
+    assert _scan(lib, _args(**kw)) == _abi.STATUS_CODE[status]
+    assert lib.ssm_last_error_detail()
+
+
+def test_scan_args_layout_matches_header(tmp_path):
+    """The ctypes mirror has the C struct's size and field offsets (compiled with gcc)."""
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    names = [f[0] for f in _abi.ScanArgs._fields_]
+    body = "\n".join(f'printf("%zu\\n", offsetof(ssm_scan_args_t, {n}));' for n in names)
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"ssm.h\"\n"
+                   "int main(void) {\n" + body +
+                   '\nprintf("%zu\\n", sizeof(ssm_scan_args_t));\nreturn 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
+    want = [getattr(_abi.ScanArgs, n).offset for n in names] + [ctypes.sizeof(_abi.ScanArgs)]
+    assert got == want
 
 
 def test_scan_args_null(lib):
