@@ -223,6 +223,13 @@ SSM_API ssm_status_t ssm_selective_scan_fwd_noalloc(const ssm_scan_args_t* args,
  * Synchronises `stream`. */
 SSM_API ssm_status_t ssm_device_error(int32_t* code, ssm_stream_t stream);
 
+/* Self-test of the failure path (the pages have no counterpart): enqueues one thread
+ * that waits, with the kernels' bounded-wait routine, on a barrier nothing completes.
+ * After limit_ns (1e3 .. 1e9, else SSM_ERR_BAD_SHAPE) the wait gives up, sets the
+ * device error word to 1 and the kernel returns; ssm_device_error() then reports it
+ * and the context stays usable. */
+SSM_API ssm_status_t ssm_wait_selftest(uint64_t limit_ns, ssm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

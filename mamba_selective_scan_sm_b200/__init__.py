@@ -20,7 +20,7 @@ from . import _abi
 from ._abi import LibraryMissing, SSMError, ScanArgs  # noqa: F401
 
 __all__ = ["ssm_causal_conv1d_fwd", "ssm_selective_scan_fwd", "ssm_selective_scan_workspace_size",
-           "ssm_selective_state_update", "ssm_device_error", "LibraryMissing", "SSMError"]
+           "ssm_selective_state_update", "ssm_device_error", "LibraryMissing", "SSMError", "ssm_wait_selftest"]
 
 
 def _torch():
@@ -188,3 +188,10 @@ def ssm_device_error(stream=None) -> int:
     code = ctypes.c_int32()
     _abi.check(lib, lib.ssm_device_error(ctypes.byref(code), _stream(stream)))
     return code.value
+
+
+def ssm_wait_selftest(limit_ns=1_000_000, stream=None) -> None:
+    """Enqueue the failure-path self-test: one bounded wait that runs out after
+    ``limit_ns`` and sets the device error word (read it with ssm_device_error)."""
+    lib = _abi.load()
+    _abi.check(lib, lib.ssm_wait_selftest(int(limit_ns), _stream(stream)))

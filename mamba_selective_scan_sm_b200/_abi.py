@@ -19,7 +19,7 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTS = (
     "ssm_abi_version", "ssm_status_string", "ssm_last_error_detail", "ssm_causal_conv1d_fwd",
     "ssm_selective_scan_workspace_size", "ssm_selective_scan_fwd", "ssm_selective_state_update",
-    "ssm_device_error", "ssm_selective_scan_fwd_noalloc",
+    "ssm_device_error", "ssm_selective_scan_fwd_noalloc", "ssm_wait_selftest",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 ABI_VERSION = 2            # SSM_ABI_VERSION of include/ssm.h this mirror follows
@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _P]
     lib.ssm_device_error.restype = ctypes.c_int
     lib.ssm_device_error.argtypes = [ctypes.POINTER(_I32), _P]
+    lib.ssm_wait_selftest.restype = ctypes.c_int
+    lib.ssm_wait_selftest.argtypes = [ctypes.c_uint64, _P]
     if lib.ssm_abi_version() != ABI_VERSION:
         raise LibraryMissing(f"{path} implements ABI {lib.ssm_abi_version()}, this binding "
                              f"expects {ABI_VERSION}: rebuild the library")

@@ -145,6 +145,21 @@ cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_
     return cudaGetLastError();
 }
 
+// One thread waits, bounded by limit_ns, on an mbarrier that nothing arrives at: the
+// wait runs out, sets the device error word and the kernel returns (a self-test of the
+// failure path every kernel's waits share).
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_bounded(&bar, 0, limit_ns);
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {
+    wait_selftest_kernel<<<1, 1, 0, st>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t read_device_error(int* code, cudaStream_t st) {
     int zero = 0;
     cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_device_error, sizeof(int), 0,

@@ -36,6 +36,9 @@ cudaError_t launch_decode(int elem_size, int dstate, const DecodeParams& p, cuda
 // Replace the calling thread's ssm_last_error_detail() text.
 void set_error_detail(const char* text);
 
+// One bounded wait that runs out after limit_ns (self-test of the failure path).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+
 // Read and clear the device error word (synchronises `stream`).
 cudaError_t read_device_error(int* code, cudaStream_t stream);
 

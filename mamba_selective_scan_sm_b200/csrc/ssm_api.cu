@@ -469,6 +469,15 @@ ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const vo
     return ok();
 }
 
+ssm_status_t ssm_wait_selftest(uint64_t limit_ns, ssm_stream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000ull)
+        return fail(SSM_ERR_BAD_SHAPE, "limit_ns %llu outside 1 us .. 1 s",
+                    (unsigned long long)limit_ns);
+    cudaError_t e = ssm::launch_wait_selftest(limit_ns, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
 ssm_status_t ssm_device_error(int32_t* code, ssm_stream_t stream) {
     if (!code) return fail(SSM_ERR_NULL_ARG, "code is NULL");
     int c = 0;

@@ -205,3 +205,9 @@ def test_device_error_null(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(_abi.LibraryMissing):
         _abi.load(str(tmp_path / "missing.so"))
+
+
+def test_wait_selftest_rejects_limits_out_of_range(lib):
+    assert lib.ssm_wait_selftest(10, None) == _abi.STATUS_CODE["SSM_ERR_BAD_SHAPE"]
+    assert lib.ssm_wait_selftest(10 ** 10, None) == _abi.STATUS_CODE["SSM_ERR_BAD_SHAPE"]
+

@@ -202,3 +202,18 @@ def test_no_device_error_after_runs():
     inp = synth.scan_inputs(1, 32, 256, 16, "bf16", conv_width=4, seed=19)
     _run(inp, "bf16", conv=True)
     assert ssm.ssm_device_error() == 0
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    """The failure path: a bounded wait on a barrier nothing completes gives up after its
+    limit (1 ms here), sets the device error word and returns; the word reads 1 once,
+    then 0, and the next scan on the same context is still correct."""
+    assert ssm.ssm_device_error() == 0
+    ssm.ssm_wait_selftest(1_000_000)
+    assert ssm.ssm_device_error() == 1
+    assert ssm.ssm_device_error() == 0
+    inp = synth.scan_inputs(1, 32, 256, 16, "bf16", conv_width=4, seed=50)
+    y, h = _run(inp, "bf16", conv=True)
+    yo, ho = _oracle(inp, conv=True)
+    assert_close_out(host(y), yo, "bf16", "y after the self-test")
+    assert ssm.ssm_device_error() == 0
