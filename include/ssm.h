@@ -153,6 +153,16 @@ typedef struct {
                                  (zeros before both) -- the conv state a decode step or
                                  the next scan continues from. Needs conv_weight; must not
                                  overlap the inputs. */
+    /* Packed sequences (batch 1, forward, no initial_state / conv_history): several
+     * sequences share the sequence axis. The state restarts from zero at every start
+     * and the fused conv reads nothing before its sequence's start. final_state is
+     * then (num_seqs, dim, dstate) and conv_state_out (num_seqs, dim, conv_width), per
+     * sequence; an empty sequence keeps zeros. */
+    const int32_t* seq_starts; /* device, num_seqs + 1 offsets: 0 = s_0 <= s_1 <= ... <=
+                                  s_num_seqs = seqlen; or NULL (one sequence per row).
+                                  Offsets out of order or range give unspecified
+                                  results (never an access outside the tensors). */
+    int32_t num_seqs;
 } ssm_scan_args_t;
 
 /* Bytes of device workspace the call with these arguments needs (0 if none).
@@ -168,8 +178,12 @@ SSM_API ssm_status_t ssm_selective_scan_workspace_size(const ssm_scan_args_t* ar
  * conv_state_out are what the next call (a scan, or ssm_selective_state_update)
  * continues from. The pages carry these two states across calls for the step method
  * (pyshine.com tour, block paragraph; paperlayer.ai §3 Method, "Autoregressive
- * cache"). Errors: SSM_ERR_UNSUPPORTED for any of initial_state, conv_history,
- * conv_state_out with reverse or the bidirectional sum; SSM_ERR_NULL_ARG for
+ * cache"). Packed sequences (seq_starts): the varlen dispatch axis of the upstream
+ * kernel (pyshine.com tour, the CUDA-core paragraph), each sequence scanned as if
+ * alone. Errors: SSM_ERR_UNSUPPORTED for any of initial_state, conv_history,
+ * conv_state_out with reverse or the bidirectional sum, and for seq_starts with
+ * batch != 1, reverse, the bidirectional sum, initial_state or conv_history;
+ * SSM_ERR_BAD_SHAPE for num_seqs < 1 with seq_starts; SSM_ERR_NULL_ARG for
  * conv_history or conv_state_out without conv_weight; SSM_ERR_ALIAS when
  * conv_state_out overlaps u, conv_history or out. */
 SSM_API ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* args, ssm_stream_t stream);

@@ -102,7 +102,8 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                            A_rev=None, D_rev=None, delta_bias_rev=None, *, out=None,
                            return_final_state=False, final_state=None, final_state_rev=None,
                            num_chunks=0, workspace=None, stream=None, initial_state=None,
-                           conv_history=None, conv_state_out=None, return_conv_state=False):
+                           conv_history=None, conv_state_out=None, return_conv_state=False,
+                           seq_starts=None):
     """Selective-scan forward (see include/ssm.h). Layouts: u, delta, z (batch, dim, seqlen);
     B, C (batch, dstate, seqlen); A (dim, dstate) fp32. With ``conv_weight`` (dim, width), ``u``
     is the pre-conv x. With ``A_rev`` the result is the bidirectional sum.
@@ -112,6 +113,9 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     sequence from ``initial_state`` (batch, dim, dstate) fp32 and ``conv_history``
     (batch, dim, width - 1); ``conv_state_out`` (batch, dim, width), allocated when
     ``return_conv_state``, receives the conv state the next call continues from.
+    ``seq_starts`` (int32, num_seqs + 1 offsets; batch 1) packs several sequences along the
+    sequence axis: final_state is then (num_seqs, dim, dstate) and the conv state
+    (num_seqs, dim, width).
     Returns ``out``, or a tuple ``(out[, final_state[, final_state_rev]][, conv_state])``.
     """
     torch = _torch()
@@ -119,21 +123,26 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     if out is None:
         out = torch.empty_like(u)
     fs, fsr = final_state, final_state_rev
+    nseq = 0 if seq_starts is None else seq_starts.numel() - 1
+    if seq_starts is not None and seq_starts.dtype != torch.int32:
+        raise TypeError("seq_starts must be int32")
+    rows = nseq if seq_starts is not None else u.shape[0]
     if return_final_state:
-        shp = (u.shape[0], u.shape[1], A.shape[1])
+        shp = (rows, u.shape[1], A.shape[1])
         if fs is None:
             fs = torch.empty(shp, dtype=torch.float32, device=u.device)
         if A_rev is not None and fsr is None:
             fsr = torch.empty(shp, dtype=torch.float32, device=u.device)
     cs = conv_state_out
     if return_conv_state and cs is None:
-        cs = torch.empty(u.shape[0], u.shape[1], conv_weight.shape[1], dtype=u.dtype,
+        cs = torch.empty(rows, u.shape[1], conv_weight.shape[1], dtype=u.dtype,
                          device=u.device)
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
                    conv_bias, A_rev, D_rev, delta_bias_rev, out, fs, fsr, num_chunks)
     a.initial_state = _fp32(initial_state, "initial_state")
     a.conv_history = _ptr(conv_history)
     a.conv_state_out = _ptr(cs)
+    a.seq_starts, a.num_seqs = _ptr(seq_starts), nseq
     n = ctypes.c_size_t()
     _abi.check(lib, lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     if n.value:

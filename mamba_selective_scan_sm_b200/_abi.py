@@ -43,6 +43,7 @@ class ScanArgs(ctypes.Structure):
         ("workspace", _P), ("workspace_bytes", ctypes.c_size_t),
         ("num_chunks", _I32),
         ("initial_state", _P), ("conv_history", _P), ("conv_state_out", _P),
+        ("seq_starts", _P), ("num_seqs", _I32),
     ]
 
 

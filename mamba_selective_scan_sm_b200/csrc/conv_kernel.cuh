@@ -88,18 +88,29 @@ __global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
 
 // The conv state a scan leaves for the next call: per row, the last `width` inputs
 // of history ++ x, oldest first, zeros before both (one thread per row; a few
-// bytes per row).
+// bytes per row). Packed sequences (batch 1): per (sequence, channel), the last
+// `width` inputs of that sequence, zeros before its start.
 template <typename T>
 __global__ void __launch_bounds__(256) conv_tail_kernel(const ConvTailParams p) {
-    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (row >= p.rows) return;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int W = p.width, L = p.seqlen;
+    int64_t row = idx;
+    int lo = 0, hi = L;                                // the row's sequence [lo, hi)
+    if (p.cu) {
+        if (idx >= (int64_t)p.nseq * p.dim) return;
+        const int s = (int)(idx / p.dim);
+        row = idx % p.dim;
+        hi = min(max(p.cu[s + 1], 0), L);             // offsets clamped into [0, L]
+        lo = min(max(p.cu[s], 0), hi);
+    } else if (idx >= p.rows) {
+        return;
+    }
     const T* x = static_cast<const T*>(p.x) + row * L;
     const T* h = p.hist ? static_cast<const T*>(p.hist) + row * (W - 1) : nullptr;
-    T* o = static_cast<T*>(p.out) + row * W;
+    T* o = static_cast<T*>(p.out) + idx * W;
     for (int k = 0; k < W; ++k) {
-        const int t = L - W + k;                       // position in the sequence
-        o[k] = t >= 0 ? x[t] : (h && t >= -(W - 1) ? h[W - 1 + t] : T(0.f));
+        const int t = hi - W + k;                      // position in the sequence axis
+        o[k] = t >= lo ? x[t] : (h && t >= -(W - 1) ? h[W - 1 + t] : T(0.f));
     }
 }
 

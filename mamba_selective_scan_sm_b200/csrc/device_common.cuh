@@ -170,9 +170,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // that lasts this long means the copy will not complete.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 
-// Device-side error word (read and cleared by ssm_device_error()). Defined here:
-// exactly one translation unit (kernels.cu) includes the device headers.
-__device__ int g_device_error = 0;
+// Device-side error word of this translation unit, set when a bounded wait runs out.
+// Every unit that includes the device headers names its own (SSM_ERROR_WORD) and
+// ssm_device_error() reads and clears them all.
+#ifndef SSM_ERROR_WORD
+#error "define SSM_ERROR_WORD (this unit's device error word) before the device headers"
+#endif
+__device__ int SSM_ERROR_WORD = 0;
 
 // Arrive on an mbarrier (release semantics at CTA scope).
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -222,7 +226,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (globaltimer_ns() - t0 > limit_ns) {
-            atomicExch(&g_device_error, 1);
+            atomicExch(&SSM_ERROR_WORD, 1);
             return false;
         }
     }

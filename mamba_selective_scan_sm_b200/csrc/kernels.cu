@@ -1,9 +1,12 @@
-// Device code of the library: one translation unit holding every kernel, the
-// device error word and the host launchers that pick a template variant.
+// Device code of the library: the conv, decode and self-test kernels, the choice of
+// scan variant and the dispatch to the scan units (scan_bf16.cu, scan_f32.cu, which
+// hold the scan kernels' instantiations and compile in parallel with this one).
+#define SSM_ERROR_WORD g_error_main
 #include "conv_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "launch.h"
 #include "scan_kernel.cuh"
+#include "scan_variants.h"
 
 namespace ssm {
 
@@ -13,26 +16,6 @@ template <typename T, int NP, int S, int KC, int SW>
 ScanVariant variant_of() {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
     return ScanVariant{(int)sizeof(T), NP, S, KC, SW, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM};
-}
-
-template <typename T, int NP, int S, int KC, int SW, bool TMA, bool SUM>
-cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
-    using Cfg = ScanCfg<T, NP, S, KC, SW>;
-    auto* k = scan_fwd_kernel<T, NP, S, KC, SW, TMA, SUM>;
-    static const cudaError_t attr =
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (attr != cudaSuccess) return attr;
-    k<<<grid, Cfg::NT, Cfg::SMEM, st>>>(maps, p);
-    return cudaGetLastError();
-}
-
-template <typename T, int NP, int S, int KC, int SW>
-cudaError_t launch_t(bool tma, bool sum, const ScanMaps& maps, const ScanParams& p, dim3 grid,
-                     cudaStream_t st) {
-    if (tma) return sum ? launch_one<T, NP, S, KC, SW, true, true>(maps, p, grid, st)
-                        : launch_one<T, NP, S, KC, SW, true, false>(maps, p, grid, st);
-    return sum ? launch_one<T, NP, S, KC, SW, false, true>(maps, p, grid, st)
-               : launch_one<T, NP, S, KC, SW, false, false>(maps, p, grid, st);
 }
 
 template <typename T, int W>
@@ -48,17 +31,6 @@ cudaError_t launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t st) {
 
 }  // namespace
 
-// (states per lane, lanes per channel, channels per lane, scan warps per CTA)
-#ifndef SSM_SCAN_VARIANTS
-#define SSM_SCAN_VARIANTS(X) \
-    X(4, 4, 1, 4)            \
-    X(4, 4, 2, 2)            \
-    X(2, 8, 1, 2)            \
-    X(2, 8, 2, 4)            \
-    X(2, 4, 1, 4)            \
-    X(1, 4, 1, 4)
-#endif
-
 bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
 #define X(NP_, S_, KC_, SW_)                                                \
     if (np == NP_ && s == S_ && kc == KC_ && sw == SW_) {                   \
@@ -71,16 +43,10 @@ bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
     return false;
 }
 
-cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
+cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, bool vl, const ScanMaps& maps,
                         const ScanParams& p, dim3 grid, cudaStream_t st) {
-#define X(NP_, S_, KC_, SW_)                                                              \
-    if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                           \
-        return v.elem_size == 2                                                           \
-                   ? launch_t<__nv_bfloat16, NP_, S_, KC_, SW_>(tma, sum, maps, p, grid, st) \
-                   : launch_t<float, NP_, S_, KC_, SW_>(tma, sum, maps, p, grid, st);
-    SSM_SCAN_VARIANTS(X)
-#undef X
-    return cudaErrorInvalidValue;
+    return v.elem_size == 2 ? launch_scan_bf16(v, tma, sum, vl, maps, p, grid, st)
+                            : launch_scan_f32(v, tma, sum, vl, maps, p, grid, st);
 }
 
 cudaError_t launch_conv_tail(int es, const ConvTailParams& p, cudaStream_t st) {
@@ -160,14 +126,22 @@ cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t read_device_error(int* code, cudaStream_t st) {
+cudaError_t take_error_main(int* code, cudaStream_t st) {
     int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_device_error, sizeof(int), 0,
+    cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_error_main, sizeof(int), 0,
                                               cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return e;
-    e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return e;
-    return cudaStreamSynchronize(st);
+    return cudaMemcpyToSymbolAsync(g_error_main, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+}
+
+cudaError_t read_device_error(int* code, cudaStream_t st) {
+    int w[3] = {0, 0, 0};
+    cudaError_t e = take_error_main(&w[0], st);
+    if (e == cudaSuccess) e = take_error_scan_bf16(&w[1], st);
+    if (e == cudaSuccess) e = take_error_scan_f32(&w[2], st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    *code = w[0] | w[1] | w[2];
+    return e;
 }
 
 }  // namespace ssm

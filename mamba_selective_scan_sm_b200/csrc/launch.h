@@ -24,8 +24,8 @@ struct ScanVariant {
 // Returns false if (elem_size, np, s, kc, sw) has no compiled kernel.
 bool scan_variant(int elem_size, int np, int s, int kc, int sw, ScanVariant* v);
 
-cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, const ScanMaps& maps,
-                        const ScanParams& p, dim3 grid, cudaStream_t stream);
+cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, bool packed,
+                        const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t stream);
 
 cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream_t stream);
 

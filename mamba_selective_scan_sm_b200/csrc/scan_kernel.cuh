@@ -25,6 +25,13 @@
 // bandwidth together; serving KC channels per lane cuts the bytes each lane reads
 // per update.
 //
+// Packed sequences (VL): several sequences share the sequence axis of one batch row,
+// starting at the offsets p.cu (p.cu[0] = 0, p.cu[nseq] = L). The state restarts from
+// zero at every start, the fused conv reads nothing before its sequence's start, and
+// each sequence's final state is written when its last step is done. One producer
+// thread finds the starts near each tile with a binary search over p.cu and stages
+// them as a bit mask with the tile.
+//
 // Two-pass chunk carry (paperlayer.ai summary of arXiv 2603.09555, §3 Method,
 // "Chunked recurrence"): with nchunks > 1, a SUMMARY launch scans every chunk but
 // the last from a zero state and writes (prod dA, h_end) per state; the output
@@ -84,7 +91,9 @@ struct ScanCfg {
     static constexpr int BUF_E = (G / KC) * P_PITCH;
     static constexpr int BUF_BT = BUF_E + G * E_PITCH;
     static constexpr int BUF_CT = BUF_BT + TT * NS * 4;
-    static constexpr int BUF = align_up(BUF_CT + TT * NS * 4, 128);
+    // packed sequences: starts at positions [l0 - HALO, l0 + TT], bit i <-> l0 - HALO + i
+    static constexpr int BUF_META = BUF_CT + TT * NS * 4;
+    static constexpr int BUF = align_up(BUF_META + 16, 128);
     static constexpr int OFF_BUF = NSTAGE * STAGE;
     static constexpr int OFF_PAR = OFF_BUF + NBUF * BUF;   // [2 directions][G][16] floats
     static constexpr int OFF_BAR = align_up(OFF_PAR + 2 * G * 64, 8);
@@ -96,6 +105,7 @@ struct ScanCfg {
     static_assert(BUF_E % 16 == 0 && BUF_BT % 16 == 0 && BUF % 16 == 0, "16-byte aligned parts");
     static_assert(NS <= 16, "at most 16 states");
     static_assert(KC == 1 || KC == 2, "one or two channels per lane");
+    static_assert(HALO + TT + 1 <= 64, "the packed-sequence window mask is 64 bits");
 };
 
 // Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 64-B
@@ -143,6 +153,14 @@ struct LaneState {
         for (int k = 0; k < NPR; ++k) { h2[k] = pk2(0.f, 0.f); pr2[k] = pk2(1.f, 1.f); }
         h1 = 0.f;
         pr1 = 1.f;
+    }
+    // A sequence starts: the state restarts from zero and no longer depends on the
+    // state carried in (the chunk product drops to zero).
+    __device__ __forceinline__ void cut() {
+#pragma unroll
+        for (int k = 0; k < NPR; ++k) { h2[k] = pk2(0.f, 0.f); pr2[k] = pk2(0.f, 0.f); }
+        h1 = 0.f;
+        pr1 = 0.f;
     }
     __device__ __forceinline__ float get(int k) const {       // k is a compile-time index
         if (ODD && k == NP - 1) return h1;
@@ -222,7 +240,7 @@ __device__ __noinline__ void put_conv_history(const ScanParams& p, uint8_t* raw_
     fence_proxy_async_smem();                     // before the stage's next TMA write
 }
 
-template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY>
+template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY, bool VL>
 __global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
@@ -354,6 +372,25 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             }
         };
 
+        // Packed sequences: the starts at positions [l0 - HALO, l0 + TT] of (forward) tile f
+        // as a bit mask (one thread).
+        auto stage_starts = [&](int f, uint8_t* buf) {
+            const int l0 = tile_l0(f);
+            const int lo = l0 - HALO;
+            int a = 0, z = p.nseq;                    // first i with cu[i] >= lo
+            while (a < z) {
+                const int m = (a + z) >> 1;
+                if (p.cu[m] < lo) a = m + 1; else z = m;
+            }
+            uint64_t wm = 0;
+            for (int i = a; i <= p.nseq && i < a + 2 * (TT + HALO + 2); ++i) {
+                const int s = p.cu[i];
+                if (s > l0 + TT) break;
+                if (s >= lo) wm |= 1ull << (s - lo);
+            }
+            *reinterpret_cast<uint64_t*>(buf + Cfg::BUF_META) = wm;
+        };
+
         // Raw stage `st` of tile f -> staging buffer `buf`. Each producer thread owns a
         // segment of SEG consecutive steps of one channel row: it reads its window of x
         // (with the conv history), dt and z with 16-byte loads, keeps the channel's
@@ -396,6 +433,12 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const uint64_t D2 = pk2(__uint_as_float(qd.x), __uint_as_float(qd.y));
             // P rows hold KC channels side by side: this channel's {delta, delta*u} slot
             uint8_t* prow_base = buf + Cfg::BUF_P + (r / KC) * Cfg::P_PITCH + (r % KC) * 8;
+            // packed sequences: the conv of step ti reads no position before its start
+            const uint64_t wm = VL ? *reinterpret_cast<const uint64_t*>(buf + Cfg::BUF_META) : 0;
+            auto first_tap = [&](int ti) {            // first tap at or after the start
+                const uint32_t w4 = (uint32_t)(wm >> (HALO + ti - 3)) & 0xFu;
+                return w4 ? 31 - __clz(w4) : 0;
+            };
 #pragma unroll
             for (int s0 = t0; s0 < t0 + SEG; s0 += SUB) {
                 // x window: row elements [s0, s0 + NXC*EPC). Forward rows start HALO steps
@@ -422,10 +465,16 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     if constexpr (CONV) {
                         // forward: u_t = sum_k w_k x[t-3+k]; reverse: u_t = sum_k w_k x[t+3-k]
                         uint64_t acc = cb2;
+                        const int fa = VL ? first_tap(s0 + i) : 0, fb = VL ? first_tap(s0 + i + 1) : 0;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int a = RV ? i + 3 - k : HALO + i - 3 + k;
-                            acc = fma2(w2[k], pk2(chunk_elem<T>(xw, a), chunk_elem<T>(xw, a + 1)), acc);
+                            float xa = chunk_elem<T>(xw, a), xb = chunk_elem<T>(xw, a + 1);
+                            if (VL) {
+                                xa = k >= fa ? xa : 0.f;
+                                xb = k >= fb ? xb : 0.f;
+                            }
+                            acc = fma2(w2[k], pk2(xa, xb), acc);
                         }
                         u2 = silu2(acc);
                     } else {
@@ -486,8 +535,10 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 // stage 0 was released by every producer at the end of tile f - 1
                 load_plain(f);
             }
+            if (VL && ptid == 0) stage_starts(f, buf_of(f));
             // one decision for all producers (this is also the barrier that orders the
-            // plain loads before the prologue): leave together if a wait ran out
+            // plain loads and the start mask before the prologue): leave together if a
+            // wait ran out
             if (named_bar_or(kProBarrier, kProThreads, !ok)) {
                 if (USE_TMA && ptid == 0)     // drain the copies still in flight (bounded)
                     for (int g2 = f; g2 < min(f + NSTAGE, nt); ++g2)
@@ -654,6 +705,29 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         const int nvalid = FULL ? TT : min(TT, ce - i0);
         const int l0 = RV ? L - i0 - TT : i0;
         const uint8_t* Prow = buf + Cfg::BUF_P + lg * Cfg::P_PITCH;
+        // packed sequences: bit tt <-> step tt starts / ends a sequence
+        const uint64_t wm = VL ? *reinterpret_cast<const uint64_t*>(buf + Cfg::BUF_META) : 0;
+        const uint32_t starts = (uint32_t)(wm >> HALO), ends = (uint32_t)(wm >> (HALO + 1));
+        // a sequence ended at step tt: its final state (the sequence is the last one whose
+        // start is <= l0 + tt; empty sequences share their successor's start)
+        auto seq_end = [&](int tt) {
+            const int t = l0 + tt;
+            int q = 0, r = p.nseq - 1;
+            while (q < r) {
+                const int m = (q + r + 1) >> 1;
+                if (p.cu[m] <= t) q = m; else r = m - 1;
+            }
+#pragma unroll
+            for (int k = 0; k < KC; ++k) {
+                if (chan_d(k) >= p.dim || !p.final_state[0]) continue;
+                float* fs = p.final_state[0] + ((int64_t)q * p.dim + chan_d(k)) * p.dstate;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    const int n = j * NP + i;
+                    if (n < p.dstate) fs[n] = ls[k].get(i);
+                }
+            }
+        };
         const float* Bl = reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * NP;
         const float* Cl = reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * NP;
         // {delta, delta*u} of step tt for the lane's KC channels
@@ -716,9 +790,16 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                         for (int k = 0; k < KC; ++k) in[u][k] = ls[k].prep(pd[k].x, pd[k].y, bv, cv);
                     }
 #pragma unroll
-                    for (int u = 0; u < KB; ++u)
+                    for (int u = 0; u < KB; ++u) {
+                        const int tt = RV ? TT - 1 - (blk * 16 + q0 + u) : blk * 16 + q0 + u;
+                        if (VL && ((starts >> tt) & 1u)) {
+#pragma unroll
+                            for (int k = 0; k < KC; ++k) ls[k].cut();
+                        }
 #pragma unroll
                         for (int k = 0; k < KC; ++k) acc[k][q0 + u] = ls[k].update(in[u][k]);
+                        if (VL && !SUMMARY && ((ends >> tt) & 1u)) seq_end(tt);
+                    }
                 }
             } else {
 #pragma unroll
@@ -732,9 +813,14 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                         float bv[NP], cv[NP];
                         load_p(tt, pd);
                         load_bc(tt, bv, cv);
+                        if (VL && ((starts >> tt) & 1u)) {
+#pragma unroll
+                            for (int k = 0; k < KC; ++k) ls[k].cut();
+                        }
 #pragma unroll
                         for (int k = 0; k < KC; ++k)
                             acc[k][q] = ls[k].update(ls[k].prep(pd[k].x, pd[k].y, bv, cv));
+                        if (VL && !SUMMARY && ((ends >> tt) & 1u)) seq_end(tt);
                     }
                 }
             }
@@ -758,7 +844,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 float2* sm = p.summary + (int64_t)chunk * p.batch * p.dim * NS + row * NS + j * NP;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) sm[i] = make_float2(ls[k].get_pr(i), ls[k].get(i));
-            } else if (chunk == p.nchunks - 1 && p.final_state[dir]) {
+            } else if (!VL && chunk == p.nchunks - 1 && p.final_state[dir]) {
                 float* fs = p.final_state[dir] + row * p.dstate;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {

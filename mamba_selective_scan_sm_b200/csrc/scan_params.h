@@ -38,6 +38,8 @@ struct ScanParams {
     float2* summary;        // two-pass: [nchunks-1][batch*dim][NS] {prod dA, h_end}
     const float* h0;        // (batch, dim, dstate) state before position 0, or nullptr
     const void* conv_hist;  // (batch, dim, conv_width-1) inputs before position 0, or nullptr
+    const int32_t* cu;      // packed sequences: nseq + 1 start offsets (cu[nseq] = seqlen)
+    int nseq;
     int vec_store;          // rows are 16-byte aligned: vector stores allowed
 };
 
@@ -46,9 +48,11 @@ struct ScanParams {
 struct ConvTailParams {
     const void* x;          // (rows, seqlen)
     const void* hist;       // (rows, width-1) or nullptr
-    void* out;              // (rows, width)
+    void* out;              // (rows, width); packed sequences: (nseq, dim, width)
     int64_t rows;
     int seqlen, width;
+    const int32_t* cu;      // packed sequences (batch 1): nseq + 1 start offsets, or nullptr
+    int nseq, dim;
 };
 
 // Standalone causal conv1d.

@@ -126,6 +126,16 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
                     "initial_state, conv_history and conv_state_out need a forward scan");
     if ((a->conv_history || a->conv_state_out) && !a->conv_weight)
         return fail(SSM_ERR_NULL_ARG, "conv_history / conv_state_out need conv_weight");
+    if (a->seq_starts) {
+        if (a->num_seqs < 1 || a->num_seqs > 0x3fffffff)
+            return fail(SSM_ERR_BAD_SHAPE, "num_seqs %d < 1", a->num_seqs);
+        if (a->batch != 1)
+            return fail(SSM_ERR_UNSUPPORTED, "packed sequences need batch 1 (got %lld)",
+                        (long long)a->batch);
+        if (bidir || a->reverse || a->initial_state || a->conv_history)
+            return fail(SSM_ERR_UNSUPPORTED,
+                        "packed sequences: forward scans without initial state or history");
+    }
 
     const int es = elem_size(a->dtype);
     const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
@@ -236,7 +246,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
         {a->final_state, 4, "final_state"}, {a->final_state_rev, 4, "final_state_rev"},
         {a->workspace, 16, "workspace"}, {a->initial_state, 4, "initial_state"},
         {a->conv_history, (size_t)es, "conv_history"},
-        {a->conv_state_out, (size_t)es, "conv_state_out"}};
+        {a->conv_state_out, (size_t)es, "conv_state_out"}, {a->seq_starts, 4, "seq_starts"}};
     for (auto& x : al)
         if (x.p && !aligned(x.p, x.al))
             return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", x.n, x.al);
@@ -246,10 +256,13 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
             overlap(a->out, act, a->C, bc))
             return fail(SSM_ERR_ALIAS, "out overlaps an input");
     }
+    const bool packed = a->seq_starts != nullptr;
+    // packed sequences: final state and conv state per sequence
+    const int64_t out_rows = packed ? (int64_t)a->num_seqs * a->dim : rows;
     const size_t st_bytes = (size_t)rows * a->dstate * sizeof(float);
     const int cw = a->conv_weight ? a->conv_width : 0;
     const size_t hist_bytes = cw > 0 ? (size_t)rows * (cw - 1) * es : 0;
-    const size_t tail_bytes = (size_t)rows * cw * es;
+    const size_t tail_bytes = (size_t)out_rows * cw * es;
     if (a->conv_state_out &&
         (overlap(a->conv_state_out, tail_bytes, a->u, act) ||
          overlap(a->conv_state_out, tail_bytes, a->conv_history, hist_bytes) ||
@@ -267,10 +280,18 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     // the conv state the next call continues from (independent of the scan's results)
     auto conv_tail = [&]() -> ssm_status_t {
         if (!a->conv_state_out || rows == 0) return SSM_OK;
-        ssm::ConvTailParams tp{a->u, a->conv_history, a->conv_state_out, rows, (int)a->seqlen, cw};
+        ssm::ConvTailParams tp{a->u, a->conv_history, a->conv_state_out, out_rows, (int)a->seqlen,
+                               cw, a->seq_starts, packed ? a->num_seqs : 0, (int)a->dim};
         cudaError_t e = ssm::launch_conv_tail(es, tp, s);
         return e == cudaSuccess ? SSM_OK : cuda_fail(e, "conv state launch");
     };
+    if (packed && a->final_state) {
+        // every sequence's final state is written at its last step; an empty sequence
+        // has none and keeps the zero initial state
+        const size_t fs = (size_t)out_rows * a->dstate * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(a->final_state, 0, fs, s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    }
     if (empty) {
         // zero steps: the final state is the initial state, the conv state its history
         const size_t fs = (size_t)rows * a->dstate * sizeof(float);
@@ -280,7 +301,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
                                                 cudaMemcpyDeviceToDevice, s);
                 if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
             }
-        } else if (fs && a->final_state) {
+        } else if (fs && a->final_state && !packed) {
             cudaError_t e = cudaMemsetAsync(a->final_state, 0, fs, s);
             if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
         }
@@ -322,6 +343,8 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     p.summary = pl.summary_bytes ? reinterpret_cast<float2*>(ws) : nullptr;
     p.h0 = a->initial_state;
     p.conv_hist = a->conv_weight ? a->conv_history : nullptr;
+    p.cu = a->seq_starts;
+    p.nseq = packed ? a->num_seqs : 0;
     if (bidir)
         p.partial = a->dtype == SSM_F32
                         ? static_cast<float*>(a->out)
@@ -353,11 +376,11 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     const unsigned gx = (unsigned)((a->dim + pl.v.channels - 1) / pl.v.channels);
     cudaError_t e;
     if (pl.nchunks > 1) {
-        e = ssm::launch_scan(pl.v, tma, true, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
+        e = ssm::launch_scan(pl.v, tma, true, packed, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
                              s);
         if (e != cudaSuccess) return cuda_fail(e, "summary pass launch");
     }
-    e = ssm::launch_scan(pl.v, tma, false, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
+    e = ssm::launch_scan(pl.v, tma, false, packed, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     if (ssm_status_t t = conv_tail(); t != SSM_OK) return t;
     return ok();

@@ -112,10 +112,19 @@ CONV = dict(conv_weight=FAKE + (1 << 30), conv_width=4)
      "SSM_ERR_ALIAS"),
     (dict(initial_state=FAKE + (1 << 29), final_state=FAKE + (1 << 29) + 64, num_chunks=4,
           seqlen=4096, workspace=FAKE + (1 << 31), workspace_bytes=1 << 20), "SSM_ERR_ALIAS"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3), "SSM_ERR_UNSUPPORTED"),            # batch 2
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3, batch=1, reverse=1), "SSM_ERR_UNSUPPORTED"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3, batch=1, A_rev=FAKE + (1 << 30)),
+     "SSM_ERR_UNSUPPORTED"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3, batch=1, initial_state=FAKE + (1 << 28)),
+     "SSM_ERR_UNSUPPORTED"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=0, batch=1), "SSM_ERR_BAD_SHAPE"),
+    (dict(seq_starts=FAKE + (1 << 29) + 2, num_seqs=3, batch=1), "SSM_ERR_MISALIGNED"),
 ])
 def test_scan_continuation_arguments(lib, kw, status):
     """initial_state / conv_history / conv_state_out: forward scans, a fused conv for the
-    conv ones, aligned, and outputs that do not overlap what the scan reads."""
+    conv ones, aligned, and outputs that do not overlap what the scan reads; packed
+    sequences: batch 1, forward, no initial state or history, at least one sequence."""
     assert _scan(lib, _args(**kw)) == _abi.STATUS_CODE[status]
     assert lib.ssm_last_error_detail()
 
