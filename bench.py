@@ -83,6 +83,9 @@ def algorithmic_bytes(w) -> int:
     dirs = 2 if w.bidirectional else 1
     params = w.dim * (w.dstate + 2) * 4 * dirs + (w.dim * (w.conv_width + 1) * 4 if w.conv_width else 0)
     fstate = rows * w.dstate * 4 * dirs if (w.final_state or w.bidirectional) else 0
+    if "packed" in w.extra:                       # per sequence: final state, offsets
+        nseq = len(synth.packed_lengths(L, *w.extra["packed"]))
+        fstate = nseq * w.dim * w.dstate * 4 + (nseq + 1) * 4
     return act + bc + params + fstate
 
 
@@ -199,16 +202,25 @@ class ScanWorkload:
         self.p = {k: par(k) for k in ("A", "D", "delta_bias", "conv_w", "conv_b", "A_rev", "D_rev",
                                       "delta_bias_rev")}
         self.out = torch.empty_like(self.t["u"])
-        shp = (w.batch, w.dim, w.dstate)
+        self.starts = None
+        rows = w.batch
+        if "packed" in w.extra:
+            lens = synth.packed_lengths(w.seqlen, *w.extra["packed"])
+            st = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+            self.starts = torch.from_numpy(st).to(device)
+            rows = len(lens)
+        shp = (rows, w.dim, w.dstate)
         self.fs = torch.empty(shp, device=device) if (w.final_state or w.bidirectional) else None
         self.fsr = torch.empty(shp, device=device) if w.bidirectional else None
         import mamba_selective_scan_sm_b200 as ssm
         self.ssm = ssm
         n = ssm.ssm_selective_scan_workspace_size(self.t["u"], self.p["A"],
                                                   conv_weight=self.p["conv_w"] if w.conv_width else None,
-                                                  A_rev=self.p["A_rev"], num_chunks=chunks)
+                                                  A_rev=self.p["A_rev"], num_chunks=chunks,
+                                                  seq_starts=self.starts)
         self.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
-        self.launches_per_step = 2 if chunks > 1 else 1
+        # a two-pass carry (asked for, or chosen for a small grid) adds the summary launch
+        self.launches_per_step = 2 if (n > 0 and not w.bidirectional) else 1
         self.h = None          # pinned host buffers of the end-to-end measurement
 
     def step(self, t=None):
@@ -219,7 +231,8 @@ class ScanWorkload:
             t["u"], t["delta"], p["A"], t["B"], t["C"], p["D"], t["z"], p["delta_bias"], True,
             False, p["conv_w"] if conv else None, p["conv_b"] if conv else None, p["A_rev"],
             p["D_rev"], p["delta_bias_rev"], out=self.out, num_chunks=self.chunks,
-            workspace=self.ws, final_state=self.fs, final_state_rev=self.fsr)
+            workspace=self.ws, final_state=self.fs, final_state_rev=self.fsr,
+            seq_starts=self.starts)
 
     def e2e_setup(self):
         torch = self.torch
@@ -411,6 +424,8 @@ def config_of(w, args):
                    if ab > L2_BYTES else "working set {:.0f} MB/step fits L2: L2-warm".format(ab / 1e6))
     if args.chunks:
         c["num_chunks"] = args.chunks
+    if "packed" in w.extra:
+        c["sequences"] = len(synth.packed_lengths(w.seqlen, *w.extra["packed"]))
     return c
 
 

@@ -80,7 +80,7 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, con
 
 
 def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num_chunks=0,
-                                      reverse=False):
+                                      reverse=False, seq_starts=None):
     """Workspace bytes ssm_selective_scan_fwd needs for these shapes (host-only query)."""
     lib = _abi.load()
     a = ScanArgs()
@@ -92,6 +92,8 @@ def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num
     a.conv_weight = 1 if conv_weight is not None else None
     a.conv_width = conv_weight.shape[1] if conv_weight is not None else 0
     a.num_chunks = int(num_chunks)
+    if seq_starts is not None:
+        a.seq_starts, a.num_seqs = 1, seq_starts.numel() - 1     # only its presence is read
     n = ctypes.c_size_t()
     _abi.check(lib, lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     return n.value

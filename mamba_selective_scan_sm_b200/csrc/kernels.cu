@@ -15,7 +15,8 @@ namespace {
 template <typename T, int NP, int S, int KC, int SW>
 ScanVariant variant_of() {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
-    return ScanVariant{(int)sizeof(T), NP, S, KC, SW, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM};
+    return ScanVariant{(int)sizeof(T), NP, S, KC, SW, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM,
+                       Cfg::MIN_CTAS};
 }
 
 template <typename T, int W>

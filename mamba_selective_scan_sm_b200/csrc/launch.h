@@ -19,6 +19,7 @@ struct ScanVariant {
     int tile;           // time steps per tile (128 bytes of elements)
     int halo;           // conv history elements fetched with a tile
     int smem_bytes;     // dynamic shared memory per CTA
+    int min_ctas;       // CTAs per SM the launch bounds are sized for
 };
 
 // Returns false if (elem_size, np, s, kc, sw) has no compiled kernel.

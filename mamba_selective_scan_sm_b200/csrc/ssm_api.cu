@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -98,6 +99,9 @@ int env_int(const char* name, int dflt) {
     return s ? std::atoi(s) : dflt;
 }
 
+// SMs of a B200 (the automatic chunk count sizes the grid against them).
+constexpr int kNumSMs = 148;
+
 ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
     if (!a) return fail(SSM_ERR_NULL_ARG, "args is NULL");
     if (a->dtype != SSM_F32 && a->dtype != SSM_BF16)
@@ -166,7 +170,21 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
     const int tile = pl->v.tile;
     const int64_t ntiles = (a->seqlen + tile - 1) / tile;
     int nch = a->num_chunks;
-    if (nch == 0) nch = 1;
+    if (nch == 0) {
+        // Automatic: when batch * dim gives too few CTAs to fill the SMs, split the
+        // sequence into chunks (two-pass carry) until the grid does. The summary pass
+        // costs about one more scan over all but the last chunk, so only a grid at most
+        // half as large as the SMs' CTA slots is split. Not for the bidirectional sum
+        // (one pass), nor when the final state overwrites the initial state.
+        const int64_t ctas = (a->dim + pl->v.channels - 1) / pl->v.channels * a->batch;
+        const int64_t slots = (int64_t)kNumSMs * pl->v.min_ctas;
+        const size_t stb = (size_t)a->batch * a->dim * a->dstate * sizeof(float);
+        const bool inplace = a->initial_state && a->final_state &&
+                             overlap(a->final_state, stb, a->initial_state, stb);
+        nch = 1;
+        if (!bidir && !inplace && ctas > 0 && 2 * ctas <= slots)
+            nch = (int)std::min<int64_t>(slots / ctas, 16);
+    }
     if (nch > ntiles) nch = (int)(ntiles > 0 ? ntiles : 1);
     if (nch > 65535) nch = 65535;
     const int64_t tiles_per_chunk = ntiles > 0 ? (ntiles + nch - 1) / nch : 1;

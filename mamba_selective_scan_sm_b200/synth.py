@@ -32,7 +32,7 @@ TID = {
     "u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "D": 6, "delta_bias": 7,
     "conv_w": 8, "D_rev": 9, "delta_bias_rev": 10, "state": 11, "conv_state": 12,
     "dec_x": 13, "dec_dt": 14, "dec_z": 15, "dec_B": 16, "dec_C": 17,
-    "A_rev": 18,
+    "A_rev": 18, "lengths": 19,
 }
 
 
@@ -104,7 +104,21 @@ WORKLOADS = {
                       bidirectional=True),
     "decode": Workload("decode B256 D5120 N16 bf16 x64 steps", 256, 5120, 1, 16, "bf16",
                        conv_width=4, steps=64),
+    "varlen": Workload("packed sequences B1 D1536 L32768 N16 bf16 + conv4, lengths "
+                       "log-uniform in [64, 4096]", 1, 1536, 32768, 16, "bf16", conv_width=4,
+                       final_state=True, extra={"packed": (64, 4096)}),
 }
+
+
+def packed_lengths(total: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
+    """Sequence lengths for packed-sequence workloads: log-uniform in [lo, hi], drawn
+    from their own stream until they cover `total`; the last one is cut to fit."""
+    g = rng(seed, TID["lengths"])
+    lens = []
+    while sum(lens) < total:
+        lens.append(int(round(np.exp(g.uniform(np.log(lo), np.log(hi))))))
+    lens[-1] -= sum(lens) - total
+    return np.array([n for n in lens if n > 0], dtype=np.int64)
 
 
 def _act(x: np.ndarray, dtype: str) -> np.ndarray:

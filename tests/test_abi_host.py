@@ -153,9 +153,17 @@ def test_scan_args_null(lib):
 
 def test_workspace_size_query(lib):
     n = ctypes.c_size_t()
-    a = _args()
+    a = _args(num_chunks=1)
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 0                               # single pass, one direction
+    # automatic: 2 x 64 channels in 8-channel CTAs fill few of the 148 SMs' slots, so the
+    # sequence (4 tiles of 32 steps) is split into as many chunks as it has tiles
+    a = _args()
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 3 * 2 * 64 * 16 * 8
+    a = _args(dim=9472 * 2)                           # enough channels: one pass
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 0
     a = _args(num_chunks=4, batch=1, dim=64, seqlen=4096)
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 3 * 1 * 64 * 16 * 8              # (chunks-1) x rows x states x (P, S)
