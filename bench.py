@@ -78,6 +78,8 @@ def algorithmic_bytes(w) -> int:
                 + w.dim * (w.dstate + 4 + 4) * 4)  # A, D, dt_bias, conv w/b
     rows = w.batch * w.dim
     L = w.seqlen
+    if w.extra.get("conv_only"):                  # x read, y write, taps and bias
+        return rows * L * es * 2 + w.dim * (w.conv_width + 1) * 4
     act = rows * L * es * 4                       # u (or x), delta, z read; y write
     bc = w.batch * w.dstate * L * es * 2          # B, C
     dirs = 2 if w.bidirectional else 1
@@ -90,6 +92,8 @@ def algorithmic_bytes(w) -> int:
 
 
 def exp_count(w) -> int:
+    if w.extra.get("conv_only"):
+        return w.batch * w.dim * w.seqlen         # one SiLU per output
     dirs = 2 if w.bidirectional else 1
     steps = max(w.seqlen, 1) * (w.steps if w.steps else 1)
     return w.batch * w.dim * steps * w.dstate * dirs
@@ -97,9 +101,15 @@ def exp_count(w) -> int:
 
 # ---------------------------------------------------------------- traffic --
 
+# each family: its kernel, the shared device headers, its launcher and the host code
+# that picks its variant (all of which decide what the captured launch did)
 KERNEL_SOURCES = {
-    "scan": ("scan_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu"),
-    "decode": ("decode_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu"),
+    "scan": ("scan_kernel.cuh", "device_common.cuh", "scan_params.h", "scan_launch.cuh",
+             "scan_variants.h", "scan_bf16.cu", "scan_f32.cu", "kernels.cu", "ssm_api.cu"),
+    "decode": ("decode_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
+               "ssm_api.cu"),
+    "conv": ("conv_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
+             "ssm_api.cu"),
 }
 
 
@@ -120,7 +130,8 @@ def recorded_traffic(key):
     path = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(path):
         return None
-    digest = kernel_source_digest("decode" if key.startswith("decode") else "scan")
+    kind = "decode" if key.startswith("decode") else ("conv" if key == "conv" else "scan")
+    digest = kernel_source_digest(kind)
     for line in open(path):
         f = [x.strip() for x in line.strip().strip("|").split("|")]
         if len(f) >= 3 and f[0] == key and f[2] == digest:
@@ -251,6 +262,53 @@ class ScanWorkload:
         return self.w.batch * self.w.dim * self.w.seqlen
 
 
+class ConvWorkload:
+    """The standalone causal conv1d + SiLU (ssm_causal_conv1d_fwd) on the m130 shape.
+
+    One step's 100 MB (x read, y written) would fit the 126 MB L2, so steps rotate over
+    SETS independent input/output pairs: a step's tensors were last touched SETS - 1
+    steps earlier, with ~200 MB of other traffic in between."""
+
+    SETS = 3
+
+    def __init__(self, w, device):
+        import torch
+        import mamba_selective_scan_sm_b200 as ssm
+        self.w, self.torch, self.ssm = w, torch, ssm
+        inp = synth.scan_inputs(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, w.conv_width, seed=0)
+        self.host_inp = inp
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        x = torch.from_numpy(inp["u"]).to(device).to(tdt)
+        self.xs = [x.clone() for _ in range(self.SETS)]
+        self.outs = [torch.empty_like(x) for _ in range(self.SETS)]
+        self.x, self.out = self.xs[0], self.outs[0]
+        self.cw = torch.from_numpy(inp["conv_w"]).to(device)
+        self.cb = torch.from_numpy(inp["conv_b"]).to(device)
+        self.k = 0
+        self.launches_per_step = 1
+        self.h = None
+
+    def step(self):
+        i = self.k % self.SETS
+        self.k += 1
+        self.ssm.ssm_causal_conv1d_fwd(self.xs[i], self.cw, self.cb, True, out=self.outs[i])
+
+    def e2e_setup(self):
+        self.h = self.x.cpu().pin_memory()
+        self.hout = self.torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d = self.h.numel() * self.h.element_size()
+        self.d2h = self.hout.numel() * self.hout.element_size()
+
+    def e2e_step(self):
+        i = self.k % self.SETS
+        self.xs[i].copy_(self.h, non_blocking=True)
+        self.step()
+        self.hout.copy_(self.outs[i], non_blocking=True)
+
+    def elems(self):
+        return self.w.batch * self.w.dim * self.w.seqlen
+
+
 class DecodeWorkload:
     """The decode configuration: 64 successive single-token updates of every (b, d) row.
 
@@ -334,6 +392,15 @@ def oracle_sample(w, seconds=10.0):
                 n += 256
         dt = time.perf_counter() - t0
         return n / dt, f"{n} single-token channel updates (batch 1, d_inner 256) of the decode workload", 1
+    if w.extra.get("conv_only"):
+        inp = synth.scan_inputs(1, 64, w.seqlen, w.dstate, w.dtype, w.conv_width, seed=0)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < seconds:
+            oracle.causal_conv1d(inp["u"], inp["conv_w"], inp["conv_b"], True)
+            n += 64 * w.seqlen
+        dt = time.perf_counter() - t0
+        return n / dt, f"{n // w.seqlen} channels x seqlen {w.seqlen} of the {w.name} workload", 1
     chans_per_call = 16
     inp = synth.scan_inputs(1, chans_per_call, w.seqlen, w.dstate, w.dtype, w.conv_width,
                             w.bidirectional, seed=0)
@@ -415,7 +482,10 @@ def config_of(w, args):
         c["tokens_per_step"] = w.steps
         c["launch"] = f"one CUDA graph of {w.steps} token launches per step"
     ab = algorithmic_bytes(w)
-    if w.name.startswith("decode"):
+    if w.extra.get("conv_only"):
+        c["l2"] = (f"steps rotate over {ConvWorkload.SETS} input/output pairs "
+                   f"({ConvWorkload.SETS * ab / 1e6:.0f} MB > 126 MB L2)")
+    elif w.name.startswith("decode"):
         c["l2"] = (f"state rotated over {DecodeWorkload.LAYERS} layers "
                    f"({DecodeWorkload.LAYERS * 94.5:.0f} MB of state > 126 MB L2): no step "
                    "finds its state in L2")
@@ -448,7 +518,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    wl = DecodeWorkload(w, device) if w.name.startswith("decode") else ScanWorkload(w, device, args.chunks)
+    if w.name.startswith("decode"):
+        wl = DecodeWorkload(w, device)
+    elif w.extra.get("conv_only"):
+        wl = ConvWorkload(w, device)
+    else:
+        wl = ScanWorkload(w, device, args.chunks)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -528,7 +603,7 @@ def main():
                "peak_kind": (f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
                              f"{sm_mhz:.0f} MHz (sampled SM clock)")}
         traffic = recorded_traffic(args.workload)
-        if w.name.startswith("decode"):
+        if w.name.startswith("decode") or w.extra.get("conv_only"):
             roof = dict(bound="hbm", **{k: hbm[k] for k in ("achieved", "peak", "unit", "frac")},
                         traffic=traffic, peak_kind=hbm["peak_kind"],
                         algorithmic_bytes_per_launch=ab, mean_launch_ms=mean_launch_ms, sfu=sfu)

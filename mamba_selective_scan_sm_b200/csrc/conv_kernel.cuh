@@ -2,9 +2,10 @@
 //
 // out[b,d,t] = act(bias[d] + sum_k w[d,k] * x[b,d,t-W+1+k]), x[t<0] = 0: output t
 // only sees inputs at positions <= t (qwerky.ai, "What We Built"). The op streams
-// one read and one write per element, so it is HBM-bound: each thread produces 8
-// consecutive outputs from one aligned 16-byte (bf16) or 2 x 16-byte (fp32) vector
-// plus the 3 preceding inputs, which the neighbouring thread also reads (L1 hit).
+// one read and one write per element, so it is HBM-bound: each thread produces 32
+// bytes of consecutive outputs from two aligned 16-byte loads plus the 16-byte chunk
+// before them (for the 3 preceding inputs; the neighbouring thread's chunk, an L1
+// hit), with the taps, the conv and the SiLU on packed fp32 pairs.
 #pragma once
 
 #include "device_common.cuh"
@@ -16,73 +17,75 @@ namespace ssm {
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
     using E = Elem<T>;
-    constexpr int V = 8;                                  // outputs per thread
+    constexpr int EPC = 16 / (int)sizeof(T);              // elements per 16-byte chunk
+    constexpr int V = 2 * EPC;                            // outputs per thread (32 bytes)
     const int L = p.seqlen;
-    // grid: x = chunks of 8 outputs along the row, y = row (b, d) in slabs of 65535
+    // grid: x = runs of V outputs along the row, y = row (b, d) in slabs of 65535
     const int t0 = (int)(blockIdx.x * blockDim.x + threadIdx.x) * V;
     const int64_t row = (int64_t)blockIdx.z * 65535 + blockIdx.y;
     if (t0 >= L || row >= p.rows) return;
-    const int d = (int)((uint64_t)row % (uint32_t)p.dim);
+    const int d = row < 0xffffffffll ? (int)((uint32_t)row % (uint32_t)p.dim)
+                                     : (int)(row % p.dim);
     const T* xr = static_cast<const T*>(p.x) + row * L;
     T* yr = static_cast<T*>(p.out) + row * L;
 
-    float w[4];
+    uint64_t w2[4];                                       // right-aligned taps, as pairs
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {                          // right-aligned taps
+    for (int k = 0; k < 4; ++k) {
         const int kk = k - (4 - p.width);
-        w[k] = kk >= 0 ? p.w[(int64_t)d * p.width + kk] : 0.f;
+        const float wk = kk >= 0 ? p.w[(int64_t)d * p.width + kk] : 0.f;
+        w2[k] = pk2(wk, wk);
     }
     const float bias = p.bias ? p.bias[d] : 0.f;
 
-    float xv[V + 3];                                       // x[t0-3 .. t0+V-1]
     if (VEC && t0 + V <= L) {
-        if constexpr (sizeof(T) == 2) {
-            const uint4 cur = *reinterpret_cast<const uint4*>(xr + t0);
-            const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&cur);
+        // x[t0 - EPC .. t0 + V): the chunk before (for the 3 previous inputs) and the
+        // thread's two chunks; position t0 - 3 + m is window element EPC - 3 + m
+        const uint4 win[3] = {t0 >= EPC ? *reinterpret_cast<const uint4*>(xr + t0 - EPC)
+                                        : make_uint4(0, 0, 0, 0),
+                              *reinterpret_cast<const uint4*>(xr + t0),
+                              *reinterpret_cast<const uint4*>(xr + t0 + EPC)};
+        uint32_t ob[V / 2];                               // bf16 pairs, or fp32 bits
+        float of[V];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float2 f = __bfloat1622float2(c2[m]);
-                xv[3 + 2 * m] = f.x;
-                xv[4 + 2 * m] = f.y;
+        for (int i = 0; i < V; i += 2) {                  // outputs t0 + i, t0 + i + 1
+            uint64_t acc = pk2(bias, bias);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                acc = fma2(w2[k], pk2(chunk_elem<T>(win, EPC - 3 + i + k),
+                                      chunk_elem<T>(win, EPC - 2 + i + k)), acc);
+            if (p.silu) acc = silu2(acc);
+            const float2 y = upk2(acc);
+            if constexpr (sizeof(T) == 2) {
+                __nv_bfloat162 t2 = __floats2bfloat162_rn(y.x, y.y);
+                ob[i / 2] = *reinterpret_cast<uint32_t*>(&t2);
+            } else {
+                of[i] = y.x;
+                of[i + 1] = y.y;
             }
-        } else {
-            const float4 a = *reinterpret_cast<const float4*>(xr + t0);
-            const float4 bq = *reinterpret_cast<const float4*>(xr + t0 + 4);
-            xv[3] = a.x; xv[4] = a.y; xv[5] = a.z; xv[6] = a.w;
-            xv[7] = bq.x; xv[8] = bq.y; xv[9] = bq.z; xv[10] = bq.w;
         }
-    } else {
-#pragma unroll
-        for (int m = 0; m < V; ++m) xv[3 + m] = (t0 + m < L) ? E::to_f(xr[t0 + m]) : 0.f;
+        if constexpr (sizeof(T) == 2) {
+            *reinterpret_cast<uint4*>(yr + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+            *reinterpret_cast<uint4*>(yr + t0 + EPC) = make_uint4(ob[4], ob[5], ob[6], ob[7]);
+        } else {
+            *reinterpret_cast<float4*>(yr + t0) = make_float4(of[0], of[1], of[2], of[3]);
+            *reinterpret_cast<float4*>(yr + t0 + 4) = make_float4(of[4], of[5], of[6], of[7]);
+        }
+        return;
     }
+    // ragged or unaligned rows: element by element
+    float w[4];
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
-        const int t = t0 - 3 + m;
-        xv[m] = t >= 0 ? E::to_f(xr[t]) : 0.f;
-    }
-    float y[V];
-#pragma unroll
-    for (int m = 0; m < V; ++m) {
+    for (int k = 0; k < 4; ++k) w[k] = lo2(w2[k]);
+    for (int m = 0; m < V && t0 + m < L; ++m) {
+        const int t = t0 + m;
         float acc = bias;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc = fmaf(w[k], xv[m + k], acc);
-        y[m] = p.silu ? silu(acc) : acc;
-    }
-    if (VEC && t0 + V <= L) {
-        if constexpr (sizeof(T) == 2) {
-            uint4 v;
-            __nv_bfloat162* v2 = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) v2[m] = __floats2bfloat162_rn(y[2 * m], y[2 * m + 1]);
-            *reinterpret_cast<uint4*>(yr + t0) = v;
-        } else {
-            *reinterpret_cast<float4*>(yr + t0) = make_float4(y[0], y[1], y[2], y[3]);
-            *reinterpret_cast<float4*>(yr + t0 + 4) = make_float4(y[4], y[5], y[6], y[7]);
+        for (int k = 0; k < 4; ++k) {
+            const int s = t - 3 + k;
+            if (s >= 0) acc = fmaf(w[k], E::to_f(xr[s]), acc);
         }
-    } else {
-#pragma unroll
-        for (int m = 0; m < V; ++m)
-            if (t0 + m < L) yr[t0 + m] = E::from_f(y[m]);
+        yr[t] = E::from_f(p.silu ? silu(acc) : acc);
     }
 }
 

@@ -127,6 +127,22 @@ __device__ __forceinline__ uint64_t softplus2(uint64_t x2) {
     return fma2(e, q, pk2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
 }
 
+// Element i (a compile-time index once unrolled) of a run of 16-byte chunks of T,
+// widened to fp32 (a bf16 value is the high half of an fp32 bit pattern).
+template <typename T, int N>
+__device__ __forceinline__ float chunk_elem(const uint4 (&w)[N], int i) {
+    constexpr int EPC = 16 / (int)sizeof(T);
+    const uint4 c = w[i / EPC];
+    if constexpr (sizeof(T) == 2) {
+        const int k = (i % 8) / 2;
+        const uint32_t word = k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w;
+        return __uint_as_float((i & 1) ? (word & 0xffff0000u) : (word << 16));
+    } else {
+        const int k = i % 4;
+        return __uint_as_float(k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w);
+    }
+}
+
 // ------------------------------------------------------- shared / barriers --
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

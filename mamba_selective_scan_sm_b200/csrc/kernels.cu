@@ -59,7 +59,7 @@ cudaError_t launch_conv_tail(int es, const ConvTailParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) {
-    const int64_t per_row = (p.seqlen + 7) / 8;
+    const int64_t per_row = (p.seqlen + 32 / es - 1) / (32 / es);   // 32 bytes per thread
     const unsigned bx = (unsigned)((per_row + 127) / 128);
     const unsigned by = (unsigned)(p.rows < 65535 ? p.rows : 65535);
     const int64_t bz = (p.rows + 65534) / 65535;

@@ -117,22 +117,6 @@ __device__ __forceinline__ int swz(int row, int byte_in_row) {
     return off ^ (((off >> 7) & SWZ) << 4);
 }
 
-// Element i (a compile-time index once unrolled) of a run of 16-byte chunks of T,
-// widened to fp32 (a bf16 value is the high half of an fp32 bit pattern).
-template <typename T, int N>
-__device__ __forceinline__ float chunk_elem(const uint4 (&w)[N], int i) {
-    constexpr int EPC = 16 / (int)sizeof(T);
-    const uint4 c = w[i / EPC];
-    if constexpr (sizeof(T) == 2) {
-        const int k = (i % 8) / 2;
-        const uint32_t word = k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w;
-        return __uint_as_float((i & 1) ? (word & 0xffff0000u) : (word << 16));
-    } else {
-        const int k = i % 4;
-        return __uint_as_float(k == 0 ? c.x : k == 1 ? c.y : k == 2 ? c.z : c.w);
-    }
-}
-
 // Recurrence state of one lane: NP states, held as fp32 pairs so the four
 // per-state operations (delta*A, delta*u*B, the h update and C.h) issue as packed
 // .f32x2 instructions.

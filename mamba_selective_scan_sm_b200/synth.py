@@ -104,6 +104,8 @@ WORKLOADS = {
                       bidirectional=True),
     "decode": Workload("decode B256 D5120 N16 bf16 x64 steps", 256, 5120, 1, 16, "bf16",
                        conv_width=4, steps=64),
+    "conv": Workload("causal conv1d + SiLU B8 D1536 L2048 bf16 width 4", 8, 1536, 2048, 16,
+                     "bf16", conv_width=4, extra={"conv_only": True}),
     "varlen": Workload("packed sequences B1 D1536 L32768 N16 bf16 + conv4, lengths "
                        "log-uniform in [64, 4096]", 1, 1536, 32768, 16, "bf16", conv_width=4,
                        final_state=True, extra={"packed": (64, 4096)}),
