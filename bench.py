@@ -499,6 +499,47 @@ def config_of(w, args):
     return c
 
 
+# ------------------------------------------------------------- replicas --
+# Every rank runs its own replica of the workload (the path needs no exchange between
+# GPUs); the host logic below is what ties the ranks together, and the CPU tests run it
+# under gloo.
+
+def init_ranks(backend, device=None, timeout_s=120):
+    """Join the process group (RANK / WORLD_SIZE / MASTER_* from the environment) when
+    more than one rank runs; returns the world size."""
+    import datetime
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1 and not dist.is_initialized():
+        kw = {"device_id": device} if device is not None and backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return world
+
+
+def max_over_ranks(value, device):
+    """The largest of every rank's value (each rank's timed region ends when its last
+    step does: the job's time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job throughput: the units all ranks processed over the job's time."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
+def leave_ranks():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -513,10 +554,7 @@ def main():
     import torch.distributed as dist
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
+    world = init_ranks("nccl", device)
 
     if w.name.startswith("decode"):
         wl = DecodeWorkload(w, device)
@@ -553,13 +591,10 @@ def main():
     clocks = sampler.stop()
     ms_total = t0.elapsed_time(t1)
     per_launch = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)]
-    if world > 1:
-        tt = torch.tensor([ms_total], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, device)
     ms_step = ms_total / args.steps
     elems = wl.elems()
-    value = elems * world / (ms_step * 1e-3)
+    value = job_throughput(elems, world, ms_step)
 
     # end to end: pinned host inputs -> device -> scan -> device result -> host
     e2e = None
@@ -577,11 +612,8 @@ def main():
         b.record(stream)
         barrier()
         ms = a.elapsed_time(b) / k
-        if world > 1:
-            tt = torch.tensor([ms], device=device)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
-        e2e = {"value": elems * world / (ms * 1e-3), "unit": "elems/s",
+        ms = max_over_ranks(ms, device)
+        e2e = {"value": job_throughput(elems, world, ms), "unit": "elems/s",
                "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": ms}
 
     if rank == 0:
@@ -636,9 +668,7 @@ def main():
                                     "kind": "oracle", "sample": desc,
                                     "single_core": {"value": v1, "cores": 1, "sample": desc1}}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    leave_ranks()
 
 
 if __name__ == "__main__":
