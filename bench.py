@@ -105,7 +105,8 @@ def exp_count(w) -> int:
 # that picks its variant (all of which decide what the captured launch did)
 KERNEL_SOURCES = {
     "scan": ("scan_kernel.cuh", "device_common.cuh", "scan_params.h", "scan_launch.cuh",
-             "scan_variants.h", "scan_bf16.cu", "scan_f32.cu", "kernels.cu", "ssm_api.cu"),
+             "scan_variants.h", "scan_bf16.cu", "scan_f32.cu", "scan_bf16_ext.cu",
+             "scan_f32_ext.cu", "kernels.cu", "ssm_api.cu"),
     "decode": ("decode_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
                "ssm_api.cu"),
     "conv": ("conv_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
@@ -209,10 +210,26 @@ class ScanWorkload:
         tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         act = lambda k: torch.from_numpy(inp[k]).to(device).to(tdt)
         par = lambda k: torch.from_numpy(inp[k]).to(device) if inp.get(k) is not None else None
-        self.t = {k: act(k) for k in ("u", "delta", "z", "B", "C")}
         self.p = {k: par(k) for k in ("A", "D", "delta_bias", "conv_w", "conv_b", "A_rev", "D_rev",
                                       "delta_bias_rev")}
-        self.out = torch.empty_like(self.t["u"])
+        self.cl = bool(w.extra.get("channel_last"))
+        if self.cl:
+            # the Mamba block's own tensors: x and z are the two halves of the in_proj
+            # output, B and C columns of the x_proj output (after its dt_rank columns)
+            B, D, L, N, R = w.batch, w.dim, w.seqlen, w.dstate, w.extra["dt_rank"]
+            cl = lambda k: act(k).transpose(1, 2)
+            xz = torch.cat([cl("u"), cl("z")], dim=2).contiguous()
+            xdbl = torch.zeros(B, L, R + 2 * N, dtype=tdt, device=device)
+            xdbl[..., R:R + N] = cl("B")
+            xdbl[..., R + N:] = cl("C")
+            self.base = {"xz": xz, "xdbl": xdbl, "dt": cl("delta").contiguous()}
+            self.t = {"u": xz[..., :D], "z": xz[..., D:], "delta": self.base["dt"],
+                      "B": xdbl[..., R:R + N], "C": xdbl[..., R + N:]}
+            self.out = torch.empty(B, L, D, dtype=tdt, device=device)
+        else:
+            self.t = {k: act(k) for k in ("u", "delta", "z", "B", "C")}
+            self.base = self.t
+            self.out = torch.empty_like(self.t["u"])
         self.starts = None
         rows = w.batch
         if "packed" in w.extra:
@@ -228,7 +245,7 @@ class ScanWorkload:
         n = ssm.ssm_selective_scan_workspace_size(self.t["u"], self.p["A"],
                                                   conv_weight=self.p["conv_w"] if w.conv_width else None,
                                                   A_rev=self.p["A_rev"], num_chunks=chunks,
-                                                  seq_starts=self.starts)
+                                                  seq_starts=self.starts, channel_last=self.cl)
         self.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
         # a two-pass carry (asked for, or chosen for a small grid) adds the summary launch
         self.launches_per_step = 2 if (n > 0 and not w.bidirectional) else 1
@@ -243,18 +260,19 @@ class ScanWorkload:
             False, p["conv_w"] if conv else None, p["conv_b"] if conv else None, p["A_rev"],
             p["D_rev"], p["delta_bias_rev"], out=self.out, num_chunks=self.chunks,
             workspace=self.ws, final_state=self.fs, final_state_rev=self.fsr,
-            seq_starts=self.starts)
+            seq_starts=self.starts, channel_last=self.cl)
 
     def e2e_setup(self):
         torch = self.torch
-        self.h = {k: v.cpu().pin_memory() for k, v in self.t.items()}
+        # the tensors a caller hands over (channel-last: the projection outputs whole)
+        self.h = {k: v.cpu().pin_memory() for k, v in self.base.items()}
         self.hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         self.h2d = sum(v.numel() * v.element_size() for v in self.h.values())
         self.d2h = self.hout.numel() * self.hout.element_size()
 
     def e2e_step(self):
         for k, v in self.h.items():
-            self.t[k].copy_(v, non_blocking=True)
+            self.base[k].copy_(v, non_blocking=True)
         self.step()
         self.hout.copy_(self.out, non_blocking=True)
 
@@ -496,6 +514,9 @@ def config_of(w, args):
         c["num_chunks"] = args.chunks
     if "packed" in w.extra:
         c["sequences"] = len(synth.packed_lengths(w.seqlen, *w.extra["packed"]))
+    if w.extra.get("channel_last"):
+        c["layout"] = (f"channel-last views: u, z of one (B, L, {2 * w.dim}) tensor, B, C of one "
+                       f"(B, L, {w.extra['dt_rank'] + 2 * w.dstate}) tensor")
     return c
 
 

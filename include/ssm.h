@@ -163,6 +163,16 @@ typedef struct {
                                   Offsets out of order or range give unspecified
                                   results (never an access outside the tensors). */
     int32_t num_seqs;
+    /* Channel-last activations: nonzero puts u, delta, z, out in (batch, seqlen, dim)
+     * and B, C in (batch, seqlen, dstate) instead. Each has an element stride between
+     * consecutive positions (0 = dense: dim, or dstate for B and C; otherwise at least
+     * that), so x and z can be views into one in_proj output (stride 2*dim) and B, C
+     * views into an x_proj output; consecutive batch rows are seqlen strides apart.
+     * The decode layouts, the conv history and conv_state_out are unchanged. With
+     * 16-byte aligned bases and strides of a multiple of 16 bytes the tiles arrive by
+     * TMA; otherwise by plain loads. */
+    int32_t channel_last;
+    int64_t stride_u, stride_delta, stride_z, stride_out, stride_B, stride_C;
 } ssm_scan_args_t;
 
 /* Bytes of device workspace the call with these arguments needs (0 if none).

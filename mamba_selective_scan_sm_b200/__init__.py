@@ -59,33 +59,62 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _position_stride(t, name):
+    """Channel-last (batch, seqlen, width) view: its element stride between positions.
+    The last axis must be dense and the batch rows seqlen positions apart."""
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    b, L, w = t.shape
+    if t.numel() and (t.stride(2) != 1 or (b > 1 and t.stride(0) != L * t.stride(1))):
+        raise ValueError(f"{name}: channel-last views need stride (seqlen*s, s, 1)")
+    return t.stride(1)
+
+
+def _view_ptr(t):
+    return None if t is None or not t.numel() else t.data_ptr()
+
+
 def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
                conv_bias, A_rev, D_rev, delta_bias_rev, out, final_state, final_state_rev,
-               num_chunks):
-    batch, dim, seqlen = u.shape
+               num_chunks, channel_last=False):
     a = ScanArgs()
     a.dtype = _dtype_code(u)
+    if channel_last:
+        batch, seqlen, dim = u.shape
+        a.channel_last = 1
+        a.stride_u, a.stride_delta = _position_stride(u, "u"), _position_stride(delta, "delta")
+        a.stride_z, a.stride_out = _position_stride(z, "z"), _position_stride(out, "out")
+        a.stride_B, a.stride_C = _position_stride(B, "B"), _position_stride(C, "C")
+        a.u, a.delta, a.B, a.C, a.z = (_view_ptr(t) for t in (u, delta, B, C, z))
+    else:
+        batch, dim, seqlen = u.shape
+        a.u, a.delta, a.B, a.C, a.z = _ptr(u), _ptr(delta), _ptr(B), _ptr(C), _ptr(z)
     a.batch, a.dim, a.seqlen, a.dstate = batch, dim, seqlen, A.shape[1]
-    a.u, a.delta, a.B, a.C, a.z = _ptr(u), _ptr(delta), _ptr(B), _ptr(C), _ptr(z)
     a.A, a.D, a.delta_bias = _fp32(A, "A"), _fp32(D, "D"), _fp32(delta_bias, "delta_bias")
     a.delta_softplus, a.reverse = int(bool(delta_softplus)), int(bool(reverse))
     a.conv_weight, a.conv_bias = _fp32(conv_weight, "conv_weight"), _fp32(conv_bias, "conv_bias")
     a.conv_width = conv_weight.shape[1] if conv_weight is not None else 0
     a.A_rev, a.D_rev = _fp32(A_rev, "A_rev"), _fp32(D_rev, "D_rev")
     a.delta_bias_rev = _fp32(delta_bias_rev, "delta_bias_rev")
-    a.out = _ptr(out)
+    a.out = _view_ptr(out) if channel_last else _ptr(out)
     a.final_state, a.final_state_rev = _ptr(final_state), _ptr(final_state_rev)
     a.num_chunks = int(num_chunks)
     return a
 
 
 def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num_chunks=0,
-                                      reverse=False, seq_starts=None):
+                                      reverse=False, seq_starts=None, channel_last=False):
     """Workspace bytes ssm_selective_scan_fwd needs for these shapes (host-only query)."""
     lib = _abi.load()
     a = ScanArgs()
     a.dtype = _dtype_code(u)
-    a.batch, a.dim, a.seqlen = u.shape
+    if channel_last:
+        a.batch, a.seqlen, a.dim = u.shape
+        a.channel_last = 1
+    else:
+        a.batch, a.dim, a.seqlen = u.shape
     a.dstate = A.shape[1]
     a.reverse = int(bool(reverse))
     a.A_rev = 1 if A_rev is not None else None
@@ -105,7 +134,7 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                            return_final_state=False, final_state=None, final_state_rev=None,
                            num_chunks=0, workspace=None, stream=None, initial_state=None,
                            conv_history=None, conv_state_out=None, return_conv_state=False,
-                           seq_starts=None):
+                           seq_starts=None, channel_last=False):
     """Selective-scan forward (see include/ssm.h). Layouts: u, delta, z (batch, dim, seqlen);
     B, C (batch, dstate, seqlen); A (dim, dstate) fp32. With ``conv_weight`` (dim, width), ``u``
     is the pre-conv x. With ``A_rev`` the result is the bidirectional sum.
@@ -117,30 +146,34 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     ``return_conv_state``, receives the conv state the next call continues from.
     ``seq_starts`` (int32, num_seqs + 1 offsets; batch 1) packs several sequences along the
     sequence axis: final_state is then (num_seqs, dim, dstate) and the conv state
-    (num_seqs, dim, width).
+    (num_seqs, dim, width). ``channel_last``: u, delta, z, out are (batch, seqlen, dim)
+    and B, C (batch, seqlen, dstate), each possibly a view with a position stride
+    (e.g. x and z halves of one in_proj output); ``out`` defaults to a dense tensor.
     Returns ``out``, or a tuple ``(out[, final_state[, final_state_rev]][, conv_state])``.
     """
     torch = _torch()
     lib = _abi.load()
     if out is None:
-        out = torch.empty_like(u)
+        out = (torch.empty(u.shape, dtype=u.dtype, device=u.device) if channel_last
+               else torch.empty_like(u))
     fs, fsr = final_state, final_state_rev
     nseq = 0 if seq_starts is None else seq_starts.numel() - 1
     if seq_starts is not None and seq_starts.dtype != torch.int32:
         raise TypeError("seq_starts must be int32")
     rows = nseq if seq_starts is not None else u.shape[0]
+    dim = u.shape[2] if channel_last else u.shape[1]
     if return_final_state:
-        shp = (rows, u.shape[1], A.shape[1])
+        shp = (rows, dim, A.shape[1])
         if fs is None:
             fs = torch.empty(shp, dtype=torch.float32, device=u.device)
         if A_rev is not None and fsr is None:
             fsr = torch.empty(shp, dtype=torch.float32, device=u.device)
     cs = conv_state_out
     if return_conv_state and cs is None:
-        cs = torch.empty(rows, u.shape[1], conv_weight.shape[1], dtype=u.dtype,
-                         device=u.device)
+        cs = torch.empty(rows, dim, conv_weight.shape[1], dtype=u.dtype, device=u.device)
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, conv_weight,
-                   conv_bias, A_rev, D_rev, delta_bias_rev, out, fs, fsr, num_chunks)
+                   conv_bias, A_rev, D_rev, delta_bias_rev, out, fs, fsr, num_chunks,
+                   channel_last)
     a.initial_state = _fp32(initial_state, "initial_state")
     a.conv_history = _ptr(conv_history)
     a.conv_state_out = _ptr(cs)

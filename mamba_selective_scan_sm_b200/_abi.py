@@ -44,6 +44,8 @@ class ScanArgs(ctypes.Structure):
         ("num_chunks", _I32),
         ("initial_state", _P), ("conv_history", _P), ("conv_state_out", _P),
         ("seq_starts", _P), ("num_seqs", _I32),
+        ("channel_last", _I32), ("stride_u", _I64), ("stride_delta", _I64), ("stride_z", _I64),
+        ("stride_out", _I64), ("stride_B", _I64), ("stride_C", _I64),
     ]
 
 

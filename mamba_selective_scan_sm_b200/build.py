@@ -9,7 +9,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libssm_b200.so")
-SOURCES = ["kernels.cu", "scan_bf16.cu", "scan_f32.cu", "ssm_api.cu", "noalloc.cu"]
+SOURCES = ["kernels.cu", "scan_bf16.cu", "scan_f32.cu", "scan_bf16_ext.cu", "scan_f32_ext.cu",
+           "ssm_api.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -108,12 +108,15 @@ __global__ void __launch_bounds__(256) conv_tail_kernel(const ConvTailParams p) 
     } else if (idx >= p.rows) {
         return;
     }
-    const T* x = static_cast<const T*>(p.x) + row * L;
+    // position t of the row: x[row * L + t], or channel-last x[(b * L + t) * stride + d]
+    const int64_t base = p.stride ? (row / p.dim) * L * p.stride + row % p.dim : row * L;
+    const int64_t step = p.stride ? p.stride : 1;
+    const T* x = static_cast<const T*>(p.x) + base;
     const T* h = p.hist ? static_cast<const T*>(p.hist) + row * (W - 1) : nullptr;
     T* o = static_cast<T*>(p.out) + idx * W;
     for (int k = 0; k < W; ++k) {
         const int t = hi - W + k;                      // position in the sequence axis
-        o[k] = t >= lo ? x[t] : (h && t >= -(W - 1) ? h[W - 1 + t] : T(0.f));
+        o[k] = t >= lo ? x[t * step] : (h && t >= -(W - 1) ? h[W - 1 + t] : T(0.f));
     }
 }
 

@@ -26,7 +26,8 @@ struct ScanVariant {
 bool scan_variant(int elem_size, int np, int s, int kc, int sw, ScanVariant* v);
 
 cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, bool packed,
-                        const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t stream);
+                        bool channel_last, const ScanMaps& maps, const ScanParams& p, dim3 grid,
+                        cudaStream_t stream);
 
 cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream_t stream);
 

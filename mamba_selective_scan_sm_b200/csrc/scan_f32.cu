@@ -1,17 +1,16 @@
-// Instantiations of the selective-scan kernel for fp32 activations (one translation
-// unit per dtype, so the variants compile in parallel).
+// Instantiations of the selective-scan kernel for fp32 activations: one sequence per row, (batch, dim, seqlen) layout.
+// (One translation unit per dtype and kind, so the variants compile in parallel.)
 #define SSM_ERROR_WORD g_error_scan_f32
 #include "scan_launch.cuh"
 #include "scan_variants.h"
 
 namespace ssm {
 
-cudaError_t launch_scan_f32(const ScanVariant& v, bool tma, bool sum, bool vl,
-                             const ScanMaps& maps, const ScanParams& p, dim3 grid,
-                             cudaStream_t st) {
-#define X(NP_, S_, KC_, SW_)                                                             \
-    if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                          \
-        return launch_t<float, NP_, S_, KC_, SW_>(tma, sum, vl, maps, p, grid, st);
+cudaError_t launch_scan_f32(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
+                             const ScanParams& p, dim3 grid, cudaStream_t st) {
+#define X(NP_, S_, KC_, SW_, EXT_)                                                          \
+    if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                            \
+        return launch_v<float, NP_, S_, KC_, SW_, false, false>(tma, sum, maps, p, grid, st);
     SSM_SCAN_VARIANTS(X)
 #undef X
     return cudaErrorInvalidValue;
@@ -22,8 +21,8 @@ cudaError_t take_error_scan_f32(int* code, cudaStream_t st) {
     cudaError_t e = cudaMemcpyFromSymbolAsync(code, g_error_scan_f32, sizeof(int), 0,
                                               cudaMemcpyDeviceToHost, st);
     if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbolAsync(g_error_scan_f32, &zero, sizeof(int), 0,
-                                   cudaMemcpyHostToDevice, st);
+    return cudaMemcpyToSymbolAsync(g_error_scan_f32, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                   st);
 }
 
 }  // namespace ssm

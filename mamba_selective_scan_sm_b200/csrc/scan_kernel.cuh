@@ -25,6 +25,15 @@
 // bandwidth together; serving KC channels per lane cuts the bytes each lane reads
 // per update.
 //
+// Channel-last activations (CL): u, delta, z, out are (batch, seqlen, dim) and B, C
+// (batch, seqlen, dstate), each with its own element stride between positions (so x
+// and z may be views into one in_proj output). The TMA boxes are then (channels x
+// steps): x/dt/z tiles land as [t][channel] and B/C tiles as [t][n], which the
+// producers only widen (no transpose); a producer reads its channel's window with
+// strided scalar loads (a warp's lanes read one row, conflict-free). The staged tile
+// is the same for both layouts, so the scan warps run the same code; only the
+// output and bidirectional-partial addresses differ.
+//
 // Packed sequences (VL): several sequences share the sequence axis of one batch row,
 // starting at the offsets p.cu (p.cu[0] = 0, p.cu[nseq] = L). The state restarts from
 // zero at every start, the fused conv reads nothing before its sequence's start, and
@@ -211,20 +220,23 @@ struct LaneState {
 // Writes the caller's conv history (the inputs at positions -(W-1) .. -1) into the
 // first forward tile's halo in shared memory. Out of line: it runs once per CTA and
 // keeps its registers out of the producer loop.
-template <typename T, int G, int HALO, int NTHR>
+template <typename T, int G, int HALO, int NTHR, bool CL>
 __device__ __noinline__ void put_conv_history(const ScanParams& p, uint8_t* raw_x, int xpitch,
                                               int ptid, int b, int d0) {
     const int hw = p.conv_width - 1;
     for (int e = ptid; e < G * hw; e += NTHR) {
         const int r = e / hw, k = e % hw, dd = d0 + r;
-        if (dd < p.dim)
-            reinterpret_cast<T*>(raw_x + r * xpitch)[HALO - hw + k] =
-                static_cast<const T*>(p.conv_hist)[((int64_t)b * p.dim + dd) * hw + k];
+        if (dd < p.dim) {
+            const T v = static_cast<const T*>(p.conv_hist)[((int64_t)b * p.dim + dd) * hw + k];
+            if (CL) reinterpret_cast<T*>(raw_x)[(HALO - hw + k) * G + r] = v;   // [t][channel]
+            else reinterpret_cast<T*>(raw_x + r * xpitch)[HALO - hw + k] = v;
+        }
     }
     fence_proxy_async_smem();                     // before the stage's next TMA write
 }
 
-template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY, bool VL>
+template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY, bool VL,
+          bool CL>
 __global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
@@ -309,15 +321,61 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 2u * NS * ROWB + G * xpitch + G * ROWB + (has_z ? G * ROWB : 0u);
             uint64_t* bar = &full_raw[f % NSTAGE];
             mbar_arrive_expect_tx(bar, bytes);
-            tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, l0, 0, b);
-            tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, l0, 0, b);
-            tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, (conv && !rv) ? l0 - HALO : l0, d0, b);
-            tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, l0, d0, b);
-            if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, l0, d0, b);
+            const int lx = (conv && !rv) ? l0 - HALO : l0;
+            if constexpr (CL) {               // maps over (channel, t, batch)
+                tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, 0, l0, b);
+                tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, 0, l0, b);
+                tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, d0, lx, b);
+                tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, d0, l0, b);
+                if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, d0, l0, b);
+            } else {                          // maps over (t, channel, batch)
+                tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, l0, 0, b);
+                tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, l0, 0, b);
+                tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, lx, d0, b);
+                tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, l0, d0, b);
+                if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, l0, d0, b);
+            }
         };
 
-        // Plain-load fallback (any alignment): fills stage 0 with the same layout.
+        // Plain-load fallback (any alignment or stride): fills stage 0 with the layout
+        // the TMA path gives.
+        auto load_plain_cl = [&](int f) {
+            uint8_t* st = smem;
+            const int l0 = tile_l0(f);
+            const bool rv = tile_rev(f);
+            const int64_t bL = (int64_t)b * L;
+            for (int e = ptid; e < NS * TT; e += kProThreads) {
+                const int n = e % NS, row = e / NS, t = l0 + row;
+                const bool ok = n < p.dstate && t >= 0 && t < L;
+                reinterpret_cast<T*>(st + Cfg::RAW_B)[e] =
+                    ok ? static_cast<const T*>(p.Bm)[(bL + t) * p.sB + n] : T(0.f);
+                reinterpret_cast<T*>(st + Cfg::RAW_C)[e] =
+                    ok ? static_cast<const T*>(p.Cm)[(bL + t) * p.sC + n] : T(0.f);
+            }
+            const int xrows = xpitch / (int)sizeof(T);
+            const int xs = (conv && !rv) ? l0 - HALO : l0;
+            const int hw = conv ? p.conv_width - 1 : 0;      // history length
+            for (int e = ptid; e < G * xrows; e += kProThreads) {
+                const int r = e % G, row = e / G, t = xs + row, dd = d0 + r;
+                const bool ok = dd < p.dim && t >= 0 && t < L;
+                const bool hist = p.conv_hist && !rv && dd < p.dim && t < 0 && t >= -hw;
+                const int64_t hi = ((int64_t)b * p.dim + dd) * hw + hw + t;
+                reinterpret_cast<T*>(st + Cfg::RAW_X)[e] =
+                    ok ? static_cast<const T*>(p.u)[(bL + t) * p.su + dd]
+                       : (hist ? static_cast<const T*>(p.conv_hist)[hi] : T(0.f));
+            }
+            for (int e = ptid; e < G * TT; e += kProThreads) {
+                const int r = e % G, row = e / G, t = l0 + row, dd = d0 + r;
+                const bool ok = dd < p.dim && t >= 0 && t < L;
+                reinterpret_cast<T*>(st + Cfg::RAW_DT)[e] =
+                    ok ? static_cast<const T*>(p.delta)[(bL + t) * p.sdl + dd] : T(0.f);
+                if (has_z)
+                    reinterpret_cast<T*>(st + Cfg::RAW_Z)[e] =
+                        ok ? static_cast<const T*>(p.z)[(bL + t) * p.sz + dd] : T(0.f);
+            }
+        };
         auto load_plain = [&](int f) {
+            if constexpr (CL) { load_plain_cl(f); return; }
             uint8_t* st = smem;
             const int l0 = tile_l0(f);
             const bool rv = tile_rev(f);
@@ -385,22 +443,41 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte chunk
             // steps per producer thread (at least one chunk; then not every thread has one)
             constexpr int SEG = TT * G / kProThreads > EPC ? TT * G / kProThreads : EPC;
-            constexpr int NSEG = TT * G / SEG;                // segments per tile
+            [[maybe_unused]] constexpr int NSEG = TT * G / SEG;   // segments per tile
             constexpr int SUB = 2 * EPC < SEG ? 2 * EPC : SEG;  // steps per register window
             constexpr int NC = SUB / EPC;                     // dt / z chunks per window
             constexpr int NXC = CONV ? NC + 1 : NC;           // x chunks (+ the conv history)
             static_assert(SEG % SUB == 0 && SUB % EPC == 0 && SUB % 2 == 0, "windows of whole chunks");
-            // B, C: swizzled [n][t] -> fp32 [t][n], one 16-byte chunk per thread and pass
+            // B, C: swizzled [n][t] -> fp32 [t][n] (channel-last: already [t][n], widened
+            // only), one 16-byte chunk per thread and pass
             constexpr int NCH = NS * ROWB / 16;               // chunks per tensor
-            for (int e = ptid; e < 2 * NCH; e += kProThreads) {
-                const int ten = e / NCH, ch = e % NCH;
-                const int n = ch % NS, c0 = (ch / NS) * EPC;
-                const uint8_t* src =
-                    st + (ten ? Cfg::RAW_C : Cfg::RAW_B) + swz<ROWB, SWZ>(n, c0 * (int)sizeof(T));
-                const uint4 v[1] = {*reinterpret_cast<const uint4*>(src)};
-                float* dst = reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) + c0 * NS + n;
+            if constexpr (CL) {
+                for (int e = ptid; e < 2 * NCH; e += kProThreads) {
+                    const int ten = e / NCH, ch = e % NCH;
+                    const uint4 v[1] = {reinterpret_cast<const uint4*>(
+                        st + (ten ? Cfg::RAW_C : Cfg::RAW_B))[ch]};
+                    float* dst = reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) +
+                                 ch * EPC;
 #pragma unroll
-                for (int m = 0; m < EPC; ++m) dst[m * NS] = chunk_elem<T>(v, m);
+                    for (int m = 0; m < EPC; m += 4)
+                        *reinterpret_cast<float4*>(dst + m) =
+                            make_float4(chunk_elem<T>(v, m), chunk_elem<T>(v, m + 1),
+                                        chunk_elem<T>(v, m + 2), chunk_elem<T>(v, m + 3));
+                }
+            } else {
+                // (braced: with an unbraced loop as the discarded branch, nvcc 12.9 also
+                // dropped the statement after it, the early return below)
+                for (int e = ptid; e < 2 * NCH; e += kProThreads) {
+                    const int ten = e / NCH, ch = e % NCH;
+                    const int n = ch % NS, c0 = (ch / NS) * EPC;
+                    const uint8_t* src = st + (ten ? Cfg::RAW_C : Cfg::RAW_B) +
+                                         swz<ROWB, SWZ>(n, c0 * (int)sizeof(T));
+                    const uint4 v[1] = {*reinterpret_cast<const uint4*>(src)};
+                    float* dst =
+                        reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) + c0 * NS + n;
+#pragma unroll
+                    for (int m = 0; m < EPC; ++m) dst[m * NS] = chunk_elem<T>(v, m);
+                }
             }
             if (NSEG < kProThreads && ptid >= NSEG) return;
             const int r = ptid % G;                           // channel row
@@ -433,14 +510,33 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     reinterpret_cast<const uint4*>(st + Cfg::RAW_DT + r * ROWB + s0 * (int)sizeof(T));
                 const uint4* zs =
                     reinterpret_cast<const uint4*>(st + Cfg::RAW_Z + r * ROWB + s0 * (int)sizeof(T));
-                uint4 xw[NXC], dw[NC], zw[NC];
+                [[maybe_unused]] uint4 xw[NXC], dw[NC], zw[NC];
+                if constexpr (!CL) {
 #pragma unroll
-                for (int c2 = 0; c2 < NXC; ++c2) xw[c2] = xs[c2];
+                    for (int c2 = 0; c2 < NXC; ++c2) xw[c2] = xs[c2];
 #pragma unroll
-                for (int c2 = 0; c2 < NC; ++c2) {
-                    dw[c2] = ds[c2];
-                    zw[c2] = has_z ? zs[c2] : make_uint4(0, 0, 0, 0);
+                    for (int c2 = 0; c2 < NC; ++c2) {
+                        dw[c2] = ds[c2];
+                        zw[c2] = has_z ? zs[c2] : make_uint4(0, 0, 0, 0);
+                    }
                 }
+                // element a of the window (raw row s0 + a of the channel): from the
+                // registers, or (channel-last) a strided load from the [t][channel] tile
+                const T* cx = reinterpret_cast<const T*>(st + Cfg::RAW_X) + r;
+                const T* cd = reinterpret_cast<const T*>(st + Cfg::RAW_DT) + r;
+                const T* cz = reinterpret_cast<const T*>(st + Cfg::RAW_Z) + r;
+                auto X = [&](int a) {
+                    if constexpr (CL) return E::to_f(cx[(s0 + a) * G]);
+                    else return chunk_elem<T>(xw, a);
+                };
+                auto DT = [&](int a) {
+                    if constexpr (CL) return E::to_f(cd[(s0 + a) * G]);
+                    else return chunk_elem<T>(dw, a);
+                };
+                auto ZV = [&](int a) {
+                    if constexpr (CL) return E::to_f(cz[(s0 + a) * G]);
+                    else return chunk_elem<T>(zw, a);
+                };
                 uint8_t* prow = prow_base + s0 * KC * 8;
                 uint8_t* erow = buf + Cfg::BUF_E + r * Cfg::E_PITCH + s0 * 8;
 #pragma unroll
@@ -453,7 +549,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int a = RV ? i + 3 - k : HALO + i - 3 + k;
-                            float xa = chunk_elem<T>(xw, a), xb = chunk_elem<T>(xw, a + 1);
+                            float xa = X(a), xb = X(a + 1);
                             if (VL) {
                                 xa = k >= fa ? xa : 0.f;
                                 xb = k >= fb ? xb : 0.f;
@@ -462,9 +558,9 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                         }
                         u2 = silu2(acc);
                     } else {
-                        u2 = pk2(chunk_elem<T>(xw, i), chunk_elem<T>(xw, i + 1));
+                        u2 = pk2(X(i), X(i + 1));
                     }
-                    uint64_t dl2 = add2(pk2(chunk_elem<T>(dw, i), chunk_elem<T>(dw, i + 1)), bias2);
+                    uint64_t dl2 = add2(pk2(DT(i), DT(i + 1)), bias2);
                     if (p.softplus) dl2 = softplus2(dl2);
                     const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
                     if constexpr (KC == 1) {
@@ -475,7 +571,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     }
                     if (!SUMMARY) {
                         uint64_t g2 = pk2(1.f, 1.f);
-                        if (has_z) g2 = silu2(pk2(chunk_elem<T>(zw, i), chunk_elem<T>(zw, i + 1)));
+                        if (has_z) g2 = silu2(pk2(ZV(i), ZV(i + 1)));
                         const float2 g = upk2(g2), dv = upk2(mul2(D2, u2));
                         *reinterpret_cast<float4*>(erow + i * 8) = make_float4(dv.x, g.x, dv.y, g.y);
                     }
@@ -513,8 +609,8 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 // The first forward tile's conv halo (positions < 0) landed as zeros;
                 // a continued sequence puts the caller's history there.
                 if (conv && p.conv_hist && p.mode == 0 && chunk == 0 && f == 0)
-                    put_conv_history<T, G, HALO, kProThreads>(p, smem + Cfg::RAW_X, xpitch, ptid,
-                                                               b, d0);
+                    put_conv_history<T, G, HALO, kProThreads, CL>(p, smem + Cfg::RAW_X, xpitch,
+                                                                   ptid, b, d0);
             } else {
                 // stage 0 was released by every producer at the end of tile f - 1
                 load_plain(f);
@@ -632,15 +728,28 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         const int mlo = rv ? R - nown : 0;
         const int mhi = rv ? R : nown;
         const int64_t gbase = chan_row(k) * L + tmin;
+        // channel-last: position t of channel d at (b*L + t) * stride + d
+        const int64_t cbase = (int64_t)b * L + tmin;
+        auto pidx = [&](int m) {
+            if constexpr (CL) return (cbase + m) * p.spart + chan_d(k);
+            else return gbase + m;
+        };
         if (p.mode == 2 && dir == 1) {
 #pragma unroll
             for (int m = 0; m < R; ++m)
-                if (m >= mlo && m < mhi) ya[m] += p.partial[gbase + m];
+                if (m >= mlo && m < mhi) ya[m] += p.partial[pidx(m)];
         }
         if (p.mode == 2 && dir == 0) {
 #pragma unroll
             for (int m = 0; m < R; ++m)
-                if (m >= mlo && m < mhi) p.partial[gbase + m] = ya[m];
+                if (m >= mlo && m < mhi) p.partial[pidx(m)] = ya[m];
+            return;
+        }
+        if constexpr (CL) {
+            T* oc = static_cast<T*>(p.out) + chan_d(k);
+#pragma unroll
+            for (int m = 0; m < R; ++m)
+                if (m >= mlo && m < mhi) oc[(cbase + m) * p.sout] = E::from_f(ya[m]);
             return;
         }
         T* out = static_cast<T*>(p.out) + gbase;

@@ -40,6 +40,8 @@ struct ScanParams {
     const void* conv_hist;  // (batch, dim, conv_width-1) inputs before position 0, or nullptr
     const int32_t* cu;      // packed sequences: nseq + 1 start offsets (cu[nseq] = seqlen)
     int nseq;
+    // channel-last activations: element strides between consecutive positions
+    int64_t su, sdl, sz, sout, sB, sC, spart;
     int vec_store;          // rows are 16-byte aligned: vector stores allowed
 };
 
@@ -53,6 +55,7 @@ struct ConvTailParams {
     int seqlen, width;
     const int32_t* cu;      // packed sequences (batch 1): nseq + 1 start offsets, or nullptr
     int nseq, dim;
+    int64_t stride;         // channel-last x: element stride between positions (0: rows of x)
 };
 
 // Standalone causal conv1d.

@@ -1,29 +1,33 @@
-// The compiled scan splits and the per-dtype scan units' entry points.
+// The compiled scan splits and the scan units' entry points.
 #pragma once
 
 #include "launch.h"
 
 namespace ssm {
 
-// (states per lane, lanes per channel, channels per lane, scan warps per CTA)
+// (states per lane, lanes per channel, channels per lane, scan warps per CTA, EXT):
+// EXT splits also have packed-sequence and channel-last kernels.
 #define SSM_SCAN_VARIANTS(X) \
-    X(4, 4, 1, 4)            \
-    X(4, 4, 2, 2)            \
-    X(2, 8, 1, 2)            \
-    X(2, 8, 2, 4)            \
-    X(2, 4, 1, 4)            \
-    X(1, 4, 1, 4)
+    X(4, 4, 1, 4, 1)         \
+    X(4, 4, 2, 2, 0)         \
+    X(2, 8, 1, 2, 1)         \
+    X(2, 8, 2, 4, 0)         \
+    X(2, 4, 1, 4, 1)         \
+    X(1, 4, 1, 4, 1)
 
-// Launch one scan pass with the split `v` (scan_bf16.cu / scan_f32.cu).
-cudaError_t launch_scan_bf16(const ScanVariant& v, bool tma, bool sum, bool packed,
-                             const ScanMaps& maps, const ScanParams& p, dim3 grid,
-                             cudaStream_t stream);
-cudaError_t launch_scan_f32(const ScanVariant& v, bool tma, bool sum, bool packed,
-                            const ScanMaps& maps, const ScanParams& p, dim3 grid,
-                            cudaStream_t stream);
-
-// Copy a unit's device error word into *code and clear it (asynchronous on `stream`).
-cudaError_t take_error_scan_bf16(int* code, cudaStream_t stream);
-cudaError_t take_error_scan_f32(int* code, cudaStream_t stream);
+// One scan pass with split `v`: one sequence per row in the (batch, dim, seqlen)
+// layout (scan_bf16.cu / scan_f32.cu), or packed sequences / channel-last
+// (scan_bf16_ext.cu / scan_f32_ext.cu).
+#define SSM_SCAN_UNIT(SUF)                                                                  \
+    cudaError_t launch_scan_##SUF(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps, \
+                                  const ScanParams& p, dim3 grid, cudaStream_t stream);       \
+    cudaError_t launch_scan_##SUF##_ext(const ScanVariant& v, bool tma, bool sum, bool packed,  \
+                                        bool channel_last, const ScanMaps& maps,              \
+                                        const ScanParams& p, dim3 grid, cudaStream_t stream); \
+    cudaError_t take_error_scan_##SUF(int* code, cudaStream_t stream);                         \
+    cudaError_t take_error_scan_##SUF##_ext(int* code, cudaStream_t stream);
+SSM_SCAN_UNIT(bf16)
+SSM_SCAN_UNIT(f32)
+#undef SSM_SCAN_UNIT
 
 }  // namespace ssm

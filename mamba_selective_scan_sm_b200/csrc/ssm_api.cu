@@ -82,6 +82,23 @@ bool encode_3d(CUtensorMap* map, int es, const void* ptr, uint64_t d0, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+// 3-D tile map with explicit byte strides of dims 1 and 2 (dim 0 innermost, dense).
+bool encode_3d_strided(CUtensorMap* map, int es, const void* ptr, uint64_t d0, uint64_t d1,
+                       uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1,
+                       CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    3, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------- scan plan --
 
 struct ScanPlan {
@@ -130,6 +147,16 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
                     "initial_state, conv_history and conv_state_out need a forward scan");
     if ((a->conv_history || a->conv_state_out) && !a->conv_weight)
         return fail(SSM_ERR_NULL_ARG, "conv_history / conv_state_out need conv_weight");
+    if (a->channel_last) {
+        struct { int64_t s, w; const char* n; } sd[] = {
+            {a->stride_u, a->dim, "stride_u"}, {a->stride_delta, a->dim, "stride_delta"},
+            {a->stride_z, a->dim, "stride_z"}, {a->stride_out, a->dim, "stride_out"},
+            {a->stride_B, a->dstate, "stride_B"}, {a->stride_C, a->dstate, "stride_C"}};
+        for (auto& x : sd)
+            if (x.s != 0 && (x.s < x.w || x.s > (1ll << 40)))
+                return fail(SSM_ERR_BAD_SHAPE, "%s %lld: 0 or at least %lld", x.n,
+                            (long long)x.s, (long long)x.w);
+    }
     if (a->seq_starts) {
         if (a->num_seqs < 1 || a->num_seqs > 0x3fffffff)
             return fail(SSM_ERR_BAD_SHAPE, "num_seqs %d < 1", a->num_seqs);
@@ -155,6 +182,7 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         if (s != 4 && s != 8) s = 4;
         kc = env_int("SSM_CHANNELS_PER_LANE", 1);
         if (kc != 1 && kc != 2) kc = 1;
+        if (a->seq_starts || a->channel_last) kc = 1;   // the splits compiled for those
         np = 16 / s;
         sw = (s == 4) == (kc == 1) ? 4 : 2;
     } else if (ns == 8) {
@@ -243,8 +271,25 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     const bool bidir = pl.mode == 2;
     const int es = elem_size(a->dtype);
     const int64_t rows = a->batch * a->dim;
+    const bool cl = a->channel_last != 0;
+    // channel-last element strides between positions (0 = dense)
+    const int64_t su = cl ? (a->stride_u ? a->stride_u : a->dim) : 0;
+    const int64_t sdl = cl ? (a->stride_delta ? a->stride_delta : a->dim) : 0;
+    const int64_t sz = cl ? (a->stride_z ? a->stride_z : a->dim) : 0;
+    const int64_t sout = cl ? (a->stride_out ? a->stride_out : a->dim) : 0;
+    const int64_t sB = cl ? (a->stride_B ? a->stride_B : a->dstate) : 0;
+    const int64_t sC = cl ? (a->stride_C ? a->stride_C : a->dstate) : 0;
+    // bytes each tensor spans: (batch, dim, seqlen) dense, or batch*seqlen positions at
+    // their stride, the last one `width` elements long
+    const int64_t npos = a->batch * a->seqlen;
+    auto span = [&](int64_t stride, int64_t width) -> size_t {
+        return npos > 0 ? (size_t)((npos - 1) * stride + width) * es : 0;
+    };
     const size_t act = (size_t)rows * a->seqlen * es;
     const size_t bc = (size_t)a->batch * a->dstate * a->seqlen * es;
+    const size_t act_u = cl ? span(su, a->dim) : act, act_dl = cl ? span(sdl, a->dim) : act;
+    const size_t act_z = cl ? span(sz, a->dim) : act, act_out = cl ? span(sout, a->dim) : act;
+    const size_t bc_B = cl ? span(sB, a->dstate) : bc, bc_C = cl ? span(sC, a->dstate) : bc;
     const bool empty = rows == 0 || a->seqlen == 0;
 
     if (!empty) {
@@ -269,9 +314,9 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
         if (x.p && !aligned(x.p, x.al))
             return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", x.n, x.al);
     if (!empty) {
-        if (overlap(a->out, act, a->u, act) || overlap(a->out, act, a->delta, act) ||
-            overlap(a->out, act, a->z, act) || overlap(a->out, act, a->B, bc) ||
-            overlap(a->out, act, a->C, bc))
+        if (overlap(a->out, act_out, a->u, act_u) || overlap(a->out, act_out, a->delta, act_dl) ||
+            overlap(a->out, act_out, a->z, act_z) || overlap(a->out, act_out, a->B, bc_B) ||
+            overlap(a->out, act_out, a->C, bc_C))
             return fail(SSM_ERR_ALIAS, "out overlaps an input");
     }
     const bool packed = a->seq_starts != nullptr;
@@ -282,9 +327,9 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     const size_t hist_bytes = cw > 0 ? (size_t)rows * (cw - 1) * es : 0;
     const size_t tail_bytes = (size_t)out_rows * cw * es;
     if (a->conv_state_out &&
-        (overlap(a->conv_state_out, tail_bytes, a->u, act) ||
+        (overlap(a->conv_state_out, tail_bytes, a->u, act_u) ||
          overlap(a->conv_state_out, tail_bytes, a->conv_history, hist_bytes) ||
-         overlap(a->conv_state_out, tail_bytes, a->out, act)))
+         overlap(a->conv_state_out, tail_bytes, a->out, act_out)))
         return fail(SSM_ERR_ALIAS, "conv_state_out overlaps u, conv_history or out");
     // one pass reads a row's initial state before writing its final state; the two-pass
     // carry reads it in every chunk while the last chunk writes the final state
@@ -299,7 +344,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     auto conv_tail = [&]() -> ssm_status_t {
         if (!a->conv_state_out || rows == 0) return SSM_OK;
         ssm::ConvTailParams tp{a->u, a->conv_history, a->conv_state_out, out_rows, (int)a->seqlen,
-                               cw, a->seq_starts, packed ? a->num_seqs : 0, (int)a->dim};
+                               cw, a->seq_starts, packed ? a->num_seqs : 0, (int)a->dim, su};
         cudaError_t e = ssm::launch_conv_tail(es, tp, s);
         return e == cudaSuccess ? SSM_OK : cuda_fail(e, "conv state launch");
     };
@@ -363,15 +408,29 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     p.conv_hist = a->conv_weight ? a->conv_history : nullptr;
     p.cu = a->seq_starts;
     p.nseq = packed ? a->num_seqs : 0;
-    if (bidir)
+    p.su = su;
+    p.sdl = sdl;
+    p.sz = sz;
+    p.sout = sout;
+    p.sB = sB;
+    p.sC = sC;
+    if (bidir) {
+        // the forward sweep's fp32 partial y: in `out` itself when fp32 (same layout and
+        // stride), else in the workspace (dense, the activations' layout)
         p.partial = a->dtype == SSM_F32
                         ? static_cast<float*>(a->out)
                         : reinterpret_cast<float*>(ws + ((pl.summary_bytes + 255) / 256) * 256);
+        p.spart = a->dtype == SSM_F32 ? sout : a->dim;
+    }
     const bool row16 = (a->seqlen * es) % 16 == 0;
-    p.vec_store = row16 && aligned(a->out, 16);
+    p.vec_store = !cl && row16 && aligned(a->out, 16);
 
-    // TMA needs 16-byte row strides and 16-byte aligned bases
-    bool tma = row16 && aligned(a->u, 16) && aligned(a->delta, 16) && aligned(a->B, 16) &&
+    // TMA needs 16-byte aligned bases and strides of a multiple of 16 bytes (and, in
+    // channel-last, B/C rows of at least 16 bytes)
+    const int ns_pad = pl.v.np * pl.v.s;
+    const bool strides16 = cl ? ((su | sdl | sz | sB | sC) * es) % 16 == 0 && ns_pad * es >= 16
+                              : row16;
+    bool tma = strides16 && aligned(a->u, 16) && aligned(a->delta, 16) && aligned(a->B, 16) &&
                aligned(a->C, 16) && (!a->z || aligned(a->z, 16)) && env_int("SSM_NO_TMA", 0) == 0;
     ssm::ScanMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -384,21 +443,35 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
         if (v.tile * es != 64) return fail(SSM_ERR_UNSUPPORTED, "tile rows must be 64 bytes");
         const CUtensorMapSwizzle bc = CU_TENSOR_MAP_SWIZZLE_64B;
         const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
-        tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
-              encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
-              (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, none)) &&
-              encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
-              encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc);
+        if (cl) {
+            // (channel, t, batch) boxes: tiles land as [t][channel] and B/C as [t][n]
+            auto map = [&](CUtensorMap* m, const void* ptr, uint64_t w, int64_t st,
+                           uint32_t b0, uint32_t b1) {
+                return encode_3d_strided(m, es, ptr, w, L, Bn, (uint64_t)st * es,
+                                         (uint64_t)st * L * es, b0, b1, none);
+            };
+            tma = map(&maps.x, a->u, D, su, v.channels, xbox) &&
+                  map(&maps.dt, a->delta, D, sdl, v.channels, v.tile) &&
+                  (!a->z || map(&maps.z, a->z, D, sz, v.channels, v.tile)) &&
+                  map(&maps.B, a->B, N, sB, ns_pad, v.tile) &&
+                  map(&maps.C, a->C, N, sC, ns_pad, v.tile);
+        } else {
+            tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
+                  encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
+                  (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, none)) &&
+                  encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
+                  encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc);
+        }
     }
 
     const unsigned gx = (unsigned)((a->dim + pl.v.channels - 1) / pl.v.channels);
     cudaError_t e;
     if (pl.nchunks > 1) {
-        e = ssm::launch_scan(pl.v, tma, true, packed, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
+        e = ssm::launch_scan(pl.v, tma, true, packed, cl, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
                              s);
         if (e != cudaSuccess) return cuda_fail(e, "summary pass launch");
     }
-    e = ssm::launch_scan(pl.v, tma, false, packed, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
+    e = ssm::launch_scan(pl.v, tma, false, packed, cl, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     if (ssm_status_t t = conv_tail(); t != SSM_OK) return t;
     return ok();

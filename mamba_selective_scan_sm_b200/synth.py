@@ -106,6 +106,10 @@ WORKLOADS = {
                        conv_width=4, steps=64),
     "conv": Workload("causal conv1d + SiLU B8 D1536 L2048 bf16 width 4", 8, 1536, 2048, 16,
                      "bf16", conv_width=4, extra={"conv_only": True}),
+    "m130_cl": Workload("Mamba-130M layer in the block's layout B8 L2048 D1536 N16 bf16 + conv4: "
+                        "x, z halves of one (B, L, 2D) in_proj output; B, C columns of one "
+                        "(B, L, 48 + 2N) x_proj output", 8, 1536, 2048, 16, "bf16", conv_width=4,
+                        extra={"channel_last": True, "dt_rank": 48}),
     "varlen": Workload("packed sequences B1 D1536 L32768 N16 bf16 + conv4, lengths "
                        "log-uniform in [64, 4096]", 1, 1536, 32768, 16, "bf16", conv_width=4,
                        final_state=True, extra={"packed": (64, 4096)}),

@@ -59,6 +59,30 @@ def test_fullsize_scan(key):
     _check(w, res, inp, chans)
 
 
+def test_fullsize_channel_last_block_layout():
+    """The Mamba-130M layer in the block's own layout (x, z halves of the in_proj output,
+    B, C columns of the x_proj output), as the benchmark times it: sampled channels
+    against the oracle, and every element equal to the (batch, dim, seqlen) call."""
+    w = synth.WORKLOADS["m130_cl"]
+    B, D, L, N, R = w.batch, w.dim, w.seqlen, w.dstate, w.extra["dt_rank"]
+    inp = synth.scan_inputs(B, D, L, N, w.dtype, w.conv_width, False, seed=0)
+    cl = lambda k: dev(inp[k], w.dtype).transpose(1, 2)
+    xz = torch.cat([cl("u"), cl("z")], dim=2).contiguous()
+    xdbl = torch.zeros(B, L, R + 2 * N, dtype=xz.dtype, device="cuda")
+    xdbl[..., R:R + N] = cl("B")
+    xdbl[..., R + N:] = cl("C")
+    f = lambda k: dev(inp[k])
+    y, h = ssm.ssm_selective_scan_fwd(
+        xz[..., :D], cl("delta").contiguous(), f("A"), xdbl[..., R:R + N], xdbl[..., R + N:],
+        f("D"), xz[..., D:], f("delta_bias"), True, False, f("conv_w"), f("conv_b"),
+        return_final_state=True, channel_last=True)
+    torch.cuda.synchronize()
+    res = (y.transpose(1, 2).contiguous(), h)
+    _check(w, res, inp, _sample(B, D, 24))
+    ref = _gpu_scan(inp, w)
+    assert torch.equal(res[0], ref[0]) and torch.equal(res[1], ref[1])
+
+
 @pytest.mark.parametrize("chunks", [0, 8])
 def test_fullsize_long_sequence(chunks):
     """65536 steps: the automatic choice and an explicit 8-chunk two-pass carry."""
