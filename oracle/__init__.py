@@ -42,7 +42,7 @@ def load_library(path: str):
     I = ctypes.c_int
     lib.oracle_causal_conv1d.argtypes = [P, P, P, P, L, L, L, I, I]
     lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, P, I, I, P, P, I, P, P, P, P,
-                                          L, L, L, L]
+                                          L, L, L, L, I]
     lib.oracle_state_update.argtypes = [P, P, P, P, P, P, P, P, P, P, I, P, P, I, P, L, L, L]
     for f in (lib.oracle_causal_conv1d, lib.oracle_selective_scan, lib.oracle_state_update):
         f.restype = None
@@ -77,31 +77,50 @@ def causal_conv1d(x, w, bias=None, apply_silu=True):
     return out
 
 
+def head_A(A, dim, N):
+    """A given per head, shape (nheads,): channel d belongs to head d // (dim // nheads)
+    and all its N states decay with that head's scalar (paperlayer.ai summary of arXiv
+    2603.09555, §3 Method, "State-space duality": A restricted to a scalar per head).
+    Returns the equivalent (dim, N) matrix; a (dim, N) A is returned unchanged."""
+    A = np.asarray(A, dtype=np.float64)
+    if A.ndim == 2:
+        return A
+    nheads = A.shape[0]
+    assert dim % nheads == 0, "dim must be a whole number of heads"
+    return np.repeat(A, dim // nheads)[:, None] * np.ones((1, N))
+
+
 def selective_scan(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                    reverse=False, conv_w=None, conv_b=None, h0=None, return_final_state=False,
                    conv_hist=None):
-    """One-direction scan. u, delta, z (B, D, L); B, C (B, N, L); A (D, N).
+    """One-direction scan. u, delta, z (B, D, L); B, C (B, N, L), or time-invariant
+    (D, N); A (D, N), or one scalar per head (nheads,).
 
     With ``conv_w`` (D, W) given, ``u`` is the pre-conv x and the scan input is
     silu(conv(x) + conv_b). ``h0`` (B, D, N) is the initial state; ``conv_hist``
     (B, D, W-1) holds the inputs before position 0, oldest first (forward only).
     Returns y (B, D, L) [and the final state (B, D, N)].
     """
-    u, delta, A, B, C = _d(u), _d(delta), _d(A), _d(B), _d(C)
+    u, delta, B, C = _d(u), _d(delta), _d(B), _d(C)
     D, z, delta_bias, conv_w, conv_b, h0 = _d(D), _d(z), _d(delta_bias), _d(conv_w), _d(conv_b), _d(h0)
     conv_hist = _d(conv_hist)
     assert conv_hist is None or (conv_w is not None and not reverse)
     Bsz, Dm, L = u.shape
-    N = A.shape[1]
-    assert delta.shape == u.shape and B.shape == (Bsz, N, L) and C.shape == (Bsz, N, L)
-    assert A.shape == (Dm, N)
+    shared = B.ndim == 2
+    N = B.shape[1]
+    A = _d(head_A(A, Dm, N))
+    if shared:
+        assert B.shape == (Dm, N) and C.shape == (Dm, N)
+    else:
+        assert B.shape == (Bsz, N, L) and C.shape == (Bsz, N, L)
+    assert delta.shape == u.shape and A.shape == (Dm, N)
     out = np.empty_like(u)
     fs = np.empty((Bsz, Dm, N), dtype=np.float64)
     W = conv_w.shape[1] if conv_w is not None else 0
     _load().oracle_selective_scan(_p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z),
                                   _p(delta_bias), int(bool(delta_softplus)), int(bool(reverse)),
                                   _p(conv_w), _p(conv_b), W, _p(h0), _p(conv_hist), _p(out),
-                                  _p(fs), Bsz, Dm, L, N)
+                                  _p(fs), Bsz, Dm, L, N, int(shared))
     return (out, fs) if return_final_state else out
 
 
@@ -154,11 +173,21 @@ def scan_channels(inp: dict, chans, *, reverse=False, conv=False, final_state=Fa
     final states (n, N) [and reverse final states for bidirectional].
     """
     ys, hs, hrs = [], [], []
+    Dm = inp["u"].shape[1]
+    shared = inp["B"].ndim == 2
+    N = inp["B"].shape[1]
     for b, d in chans:
         sl = lambda a: None if a is None else a[b:b + 1, d:d + 1]
-        args = dict(u=sl(inp["u"]), delta=sl(inp["delta"]), B=inp["B"][b:b + 1],
-                    C=inp["C"][b:b + 1], z=sl(inp.get("z")))
-        pd = lambda k: None if inp.get(k) is None else inp[k][d:d + 1]
+        bc = (lambda k: inp[k][d:d + 1]) if shared else (lambda k: inp[k][b:b + 1])
+        args = dict(u=sl(inp["u"]), delta=sl(inp["delta"]), B=bc("B"), C=bc("C"),
+                    z=sl(inp.get("z")))
+
+        def pd(k):
+            if inp.get(k) is None:
+                return None
+            if k in ("A", "A_rev"):
+                return head_A(inp[k], Dm, N)[d:d + 1]
+            return inp[k][d:d + 1]
         cw = pd("conv_w") if conv else None
         cb = pd("conv_b") if conv else None
         if bidirectional:

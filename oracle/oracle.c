@@ -36,6 +36,10 @@
  *  - the reverse final state is the state after position 0 (its last step).
  *  - decode conv state holds the last W inputs, newest last; it shifts left by one
  *    and appends x_t before the convolution.
+ *  - B and C are either input-dependent, (Bsz, N, L) and shared by all channels, or
+ *    time-invariant, (D, N): one fixed row per channel, the same at every position
+ *    (pyshine.com tour, the CUDA-core paragraph: the kernel dispatches on "whether B
+ *    and C are variable or shared"; the time-invariant form is the classic LTI SSM).
  *  - a forward scan may continue a sequence processed earlier (a prompt taken in
  *    pieces, or a prefill after decode steps): it then starts from that sequence's
  *    state h0 and its conv reads the W-1 inputs that preceded position 0 (conv_hist,
@@ -79,7 +83,8 @@ void oracle_causal_conv1d(const double* x, const double* w, const double* bias, 
 }
 
 /* Selective-scan forward (one direction).
- * u, delta, z, out: (Bsz, D, L); Bm, Cm: (Bsz, N, L); A: (D, N);
+ * u, delta, z, out: (Bsz, D, L); Bm, Cm: (Bsz, N, L), or (D, N) when bc_shared
+ * (time-invariant: channel d reads row d at every position); A: (D, N);
  * Dv, delta_bias, conv_b: (D) or NULL; conv_w: (D, W) or NULL (NULL: no conv);
  * h0: (Bsz, D, N) initial state or NULL (zeros); final_state: (Bsz, D, N) or NULL.
  * conv_hist: (Bsz, D, W-1) inputs at positions -(W-1) .. -1, oldest first, or NULL
@@ -90,7 +95,8 @@ void oracle_selective_scan(const double* u, const double* delta, const double* A
                            const double* z, const double* delta_bias, int delta_softplus,
                            int reverse, const double* conv_w, const double* conv_b,
                            int conv_width, const double* h0, const double* conv_hist,
-                           double* out, double* final_state, long Bsz, long D, long L, long N) {
+                           double* out, double* final_state, long Bsz, long D, long L, long N,
+                           int bc_shared) {
     double h[1024];
     if (N > 1024) return;
     for (long b = 0; b < Bsz; ++b)
@@ -98,8 +104,10 @@ void oracle_selective_scan(const double* u, const double* delta, const double* A
             const double* ur = u + (b * D + d) * L;
             const double* dr = delta + (b * D + d) * L;
             const double* zr = z ? z + (b * D + d) * L : NULL;
-            const double* Br = Bm + b * N * L;
-            const double* Cr = Cm + b * N * L;
+            /* B[n] at position t is Br[n * bn + t * bt] */
+            const double* Br = bc_shared ? Bm + d * N : Bm + b * N * L;
+            const double* Cr = bc_shared ? Cm + d * N : Cm + b * N * L;
+            const long bn = bc_shared ? 1 : L, bt = bc_shared ? 0 : 1;
             double* yr = out + (b * D + d) * L;
             for (long n = 0; n < N; ++n) h[n] = h0 ? h0[(b * D + d) * N + n] : 0.0;
             for (long i = 0; i < L; ++i) {
@@ -126,9 +134,9 @@ void oracle_selective_scan(const double* u, const double* delta, const double* A
                 double y = 0.0;
                 for (long n = 0; n < N; ++n) {
                     double dA = exp(dl * A[d * N + n]);
-                    double dBu = dl * Br[n * L + t] * ut;
+                    double dBu = dl * Br[n * bn + t * bt] * ut;
                     h[n] = dA * h[n] + dBu;
-                    y += Cr[n * L + t] * h[n];
+                    y += Cr[n * bn + t * bt] * h[n];
                 }
                 if (Dv) y += Dv[d] * ut;
                 if (zr) y *= silu(zr[t]);

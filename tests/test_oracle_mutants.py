@@ -7,6 +7,8 @@ fail. The committed oracle itself is untouched.
 """
 import itertools
 import os
+
+import numpy as np
 import subprocess
 import tempfile
 
@@ -25,13 +27,22 @@ MUTANTS = [
      "if (zr) y *= silu(zr[t]);\n                if (Dv) y += Dv[d] * ut;", None),
     ("decay sign flipped", "exp(dl * A[d * N + n])", "exp(-dl * A[d * N + n])", None),
     ("delta missing from the decay", "exp(dl * A[d * N + n])", "exp(A[d * N + n])", None),
-    ("delta missing from dBu", "double dBu = dl * Br[n * L + t] * ut;",
-     "double dBu = Br[n * L + t] * ut;", None),
-    ("B and C swapped", "dl * Br[n * L + t] * ut", "dl * Cr[n * L + t] * ut", None),
-    ("B read transposed", "dl * Br[n * L + t] * ut", "dl * Br[t * N + n] * ut", None),
+    ("delta missing from dBu", "double dBu = dl * Br[n * bn + t * bt] * ut;",
+     "double dBu = Br[n * bn + t * bt] * ut;", None),
+    ("B and C swapped", "dl * Br[n * bn + t * bt] * ut", "dl * Cr[n * bn + t * bt] * ut", None),
+    ("B read transposed", "dl * Br[n * bn + t * bt] * ut", "dl * Br[t * N + n] * ut", None),
     ("readout before the update",
-     "h[n] = dA * h[n] + dBu;\n                    y += Cr[n * L + t] * h[n];",
-     "y += Cr[n * L + t] * h[n];\n                    h[n] = dA * h[n] + dBu;", None),
+     "h[n] = dA * h[n] + dBu;\n                    y += Cr[n * bn + t * bt] * h[n];",
+     "y += Cr[n * bn + t * bt] * h[n];\n                    h[n] = dA * h[n] + dBu;", None),
+    ("time-invariant B read as (N, D)", "bc_shared ? Bm + d * N : Bm + b * N * L",
+     "bc_shared ? Bm + d : Bm + b * N * L", None),
+    ("time-invariant B and C read as (N, D) matrices",
+     "const double* Br = bc_shared ? Bm + d * N : Bm + b * N * L;\n"
+     "            const double* Cr = bc_shared ? Cm + d * N : Cm + b * N * L;\n"
+     "            const long bn = bc_shared ? 1 : L,",
+     "const double* Br = bc_shared ? Bm + d : Bm + b * N * L;\n"
+     "            const double* Cr = bc_shared ? Cm + d : Cm + b * N * L;\n"
+     "            const long bn = bc_shared ? D : L,", None),
     ("conv taps reversed", "long s = t - (W - 1) + k;", "long s = t - k;", None),
     ("fused conv taps reversed", ": t - (conv_width - 1) + k;", ": t - k;", None),
     ("reverse conv uses forward taps", "t + (conv_width - 1) - k :", "t - (conv_width - 1) + k :",
@@ -115,3 +126,16 @@ def test_mutant_is_caught(name, old, new, occ, tmp_path):
                            "-shared", "-fPIC", "-o", str(so), str(c), "-lm"])
     failed = _failing_pins(oracle.load_library(str(so)))
     assert failed, f"no pin caught the planted mistake: {name}"
+
+
+def test_head_mapping_slip_is_caught(monkeypatch):
+    """A plausible slip in the per-head expansion (heads interleaved across channels
+    instead of contiguous) fails the dual-form pin."""
+    def wrong(A, dim, N):
+        A = np.asarray(A, dtype=np.float64)
+        if A.ndim == 2:
+            return A
+        return np.tile(A, dim // A.shape[0])[:, None] * np.ones((1, N))
+    monkeypatch.setattr(oracle, "head_A", wrong)
+    with pytest.raises(AssertionError):
+        pins.test_scalar_A_per_head_equals_ssd_dual_form(4, False)

@@ -457,3 +457,101 @@ def test_oracle_consumes_bf16_rounded_inputs():
     big = np.random.default_rng(14).standard_normal(100000).astype(np.float32)
     np.testing.assert_array_equal(synth.round_bf16(big),
                                   torch.from_numpy(big).to(torch.bfloat16).float().numpy())
+
+
+# ------------------------------------------- heads, time-invariant B/C, large N ---
+# State-space duality (paperlayer.ai summary of arXiv 2603.09555, §3 Method, "State-space
+# duality" and "Chunked recurrence"): with A diagonal the recurrence unrolls to
+#   h_t[n] = sum_{s<=t} exp(sum_{r=s+1..t} delta_r A[n]) delta_s u_s B_s[n],
+# so y = sum_n (M_n o C[:, n] B[:, n]^T) (delta u) with the lower-triangular decay
+# matrix M_n[t, s] = exp(cum_n[t] - cum_n[s]). The pins below evaluate that quadratic
+# form with numpy matrix products: no recurrence, no loop over time.
+
+def _dual_form(u, dl, A_dn, Bt, Ct, Dv, z):
+    """One channel. u, dl, z (L,); A_dn (N,); Bt, Ct (L, N). Returns y (L,), h_L (N,)."""
+    L, N = Bt.shape
+    x = dl * u
+    tri = np.tril(np.ones((L, L), dtype=bool))
+    y = np.zeros(L)
+    hL = np.zeros(N)
+    for n in range(N):
+        cum = np.cumsum(dl * A_dn[n])
+        M = np.where(tri, np.exp(np.where(tri, cum[:, None] - cum[None, :], 0.0)), 0.0)
+        y += (M * np.outer(Ct[:, n], Bt[:, n])) @ x
+        hL[n] = (M[-1] * Bt[:, n]) @ x
+    if Dv is not None:
+        y += Dv * u
+    if z is not None:
+        y *= _silu(z)
+    return y, hL
+
+
+def _head_case(rng, Bsz, nheads, P, L, N, shared):
+    D = nheads * P
+    c = dict(u=rng.standard_normal((Bsz, D, L)), delta=0.5 * rng.standard_normal((Bsz, D, L)),
+             z=rng.standard_normal((Bsz, D, L)), A=-rng.uniform(0.2, 2.0, nheads),
+             D=rng.standard_normal(D), delta_bias=rng.uniform(-3, 0.5, D))
+    shp = (D, N) if shared else (Bsz, N, L)
+    c["B"], c["C"] = rng.standard_normal(shp), rng.standard_normal(shp)
+    return c
+
+
+def _bc_rows(c, b, d, L):
+    if c["B"].ndim == 2:                     # time-invariant: row d at every position
+        return np.tile(c["B"][d], (L, 1)), np.tile(c["C"][d], (L, 1))
+    return c["B"][b].T, c["C"][b].T
+
+
+@pytest.mark.parametrize("N,shared", [(4, False), (4, True), (64, False), (16, True)])
+def test_scalar_A_per_head_equals_ssd_dual_form(N, shared):
+    """A one scalar per head: every channel of head h decays all its states with A_h."""
+    rng = np.random.default_rng(81)
+    Bsz, nheads, P, L = 2, 3, 2, 11
+    c = _head_case(rng, Bsz, nheads, P, L, N, shared)
+    y, hf = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                  c["delta_bias"], True, return_final_state=True)
+    dl = _softplus(c["delta"] + c["delta_bias"][None, :, None])
+    for b in range(Bsz):
+        for d in range(nheads * P):
+            Bt, Ct = _bc_rows(c, b, d, L)
+            A_dn = np.full(N, c["A"][d // P])
+            yd, hd = _dual_form(c["u"][b, d], dl[b, d], A_dn, Bt, Ct, c["D"][d], c["z"][b, d])
+            np.testing.assert_allclose(y[b, d], yd, rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(hf[b, d], hd, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("N", [8, 128])
+def test_per_state_A_equals_dual_form(N):
+    """The general diagonal A (dim, N), variable B/C, at d_state up to 128."""
+    rng = np.random.default_rng(82)
+    c = _rand_case(rng, B=1, D=2, L=9, N=N)
+    y, hf = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                                  c["delta_bias"], True, return_final_state=True)
+    dl = _softplus(c["delta"] + c["delta_bias"][None, :, None])
+    for d in range(2):
+        yd, hd = _dual_form(c["u"][0, d], dl[0, d], c["A"][d], c["B"][0].T, c["C"][0].T,
+                            c["D"][d], c["z"][0, d])
+        np.testing.assert_allclose(y[0, d], yd, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(hf[0, d], hd, rtol=1e-10, atol=1e-12)
+
+
+def test_time_invariant_BC_constant_inputs_closed_form():
+    """Constant delta and u with B, C fixed per channel (the LTI case): each state is a
+    geometric series, h_t = delta u B[d, n] (1 - a^(t+1)) / (1 - a), a = exp(delta A)."""
+    rng = np.random.default_rng(83)
+    Dm, L, N = 3, 12, 5
+    A = -rng.uniform(0.1, 1.5, (Dm, N))
+    Bs, Cs = rng.standard_normal((Dm, N)), rng.standard_normal((Dm, N))
+    dl, uval = 0.37, 0.8
+    u = np.full((1, Dm, L), uval)
+    delta = np.full((1, Dm, L), dl)
+    Dv = rng.standard_normal(Dm)
+    y, hf = oracle.selective_scan(u, delta, A, Bs, Cs, Dv, None, None, False,
+                                  return_final_state=True)
+    t = np.arange(L)
+    for d in range(Dm):
+        a = np.exp(dl * A[d])                                    # (N,)
+        h = dl * uval * Bs[d][None, :] * (1 - a[None, :] ** (t[:, None] + 1)) / (1 - a[None, :])
+        np.testing.assert_allclose(y[0, d], h @ Cs[d] + Dv[d] * uval, rtol=1e-12)
+        np.testing.assert_allclose(hf[0, d], h[-1], rtol=1e-12)
+
