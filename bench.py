@@ -37,7 +37,8 @@ from mamba_selective_scan_sm_b200 import synth  # noqa: E402
 
 METRIC = "selective-scan fwd B*D*L elems/s and achieved HBM GB/s vs B200 peak (1 GPU)"
 L2_BYTES = 126 * 1024 * 1024
-SFU_EX2_PER_CLK_PER_SM = 16      # MUFU.EX2 results per clock per SM (measured: see the design doc)
+SFU_EX2_PER_CLK_PER_SM = 16      # MUFU.EX2 results per clock per SM (a standalone ex2 loop on B200)
+FP32_LANES_PER_SM = 128          # FP32 FMA lanes per SM per clock (4 SMSPs x 32)
 N_SM = 148
 
 
@@ -81,9 +82,11 @@ def algorithmic_bytes(w) -> int:
     if w.extra.get("conv_only"):                  # x read, y write, taps and bias
         return rows * L * es * 2 + w.dim * (w.conv_width + 1) * 4
     act = rows * L * es * 4                       # u (or x), delta, z read; y write
-    bc = w.batch * w.dstate * L * es * 2          # B, C
+    bc = (w.dim * w.dstate * 4 * 2 if w.extra.get("bc_shared")       # B, C fixed per channel
+          else w.batch * w.dstate * L * es * 2)   # B, C
     dirs = 2 if w.bidirectional else 1
-    params = w.dim * (w.dstate + 2) * 4 * dirs + (w.dim * (w.conv_width + 1) * 4 if w.conv_width else 0)
+    a_par = w.extra["a_heads"] if w.extra.get("a_heads") else w.dim * w.dstate
+    params = (a_par + w.dim * 2) * 4 * dirs + (w.dim * (w.conv_width + 1) * 4 if w.conv_width else 0)
     fstate = rows * w.dstate * 4 * dirs if (w.final_state or w.bidirectional) else 0
     if "packed" in w.extra:                       # per sequence: final state, offsets
         nseq = len(synth.packed_lengths(L, *w.extra["packed"]))
@@ -96,7 +99,15 @@ def exp_count(w) -> int:
         return w.batch * w.dim * w.seqlen         # one SiLU per output
     dirs = 2 if w.bidirectional else 1
     steps = max(w.seqlen, 1) * (w.steps if w.steps else 1)
-    return w.batch * w.dim * steps * w.dstate * dirs
+    per_state = 1 if w.extra.get("a_heads") else w.dstate   # A per head: one exp per step
+    return w.batch * w.dim * steps * per_state * dirs
+
+
+def fp32_ops(w) -> int:
+    """FP32 operations the recurrence cannot avoid: per state and step dBu = du * B,
+    h = dA * h + dBu (one FMA) and the readout C * h (one FMA)."""
+    dirs = 2 if w.bidirectional else 1
+    return 3 * w.batch * w.dim * max(w.seqlen, 1) * w.dstate * dirs
 
 
 # ---------------------------------------------------------------- traffic --
@@ -205,7 +216,8 @@ class ScanWorkload:
         self.torch = torch
         self.chunks = chunks
         inp = synth.scan_inputs(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, w.conv_width,
-                                w.bidirectional, seed=0)
+                                w.bidirectional, seed=0, a_heads=w.extra.get("a_heads", 0),
+                                bc_shared=bool(w.extra.get("bc_shared")))
         self.host_inp = inp
         tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         act = lambda k: torch.from_numpy(inp[k]).to(device).to(tdt)
@@ -245,7 +257,9 @@ class ScanWorkload:
         n = ssm.ssm_selective_scan_workspace_size(self.t["u"], self.p["A"],
                                                   conv_weight=self.p["conv_w"] if w.conv_width else None,
                                                   A_rev=self.p["A_rev"], num_chunks=chunks,
-                                                  seq_starts=self.starts, channel_last=self.cl)
+                                                  seq_starts=self.starts, channel_last=self.cl,
+                                                  dstate=w.dstate,
+                                                  bc_shared=bool(w.extra.get("bc_shared")))
         self.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
         # a two-pass carry (asked for, or chosen for a small grid) adds the summary launch
         self.launches_per_step = 2 if (n > 0 and not w.bidirectional) else 1
@@ -420,8 +434,10 @@ def oracle_sample(w, seconds=10.0):
         dt = time.perf_counter() - t0
         return n / dt, f"{n // w.seqlen} channels x seqlen {w.seqlen} of the {w.name} workload", 1
     chans_per_call = 16
+    # A per head: the sample's 16 channels form one head
     inp = synth.scan_inputs(1, chans_per_call, w.seqlen, w.dstate, w.dtype, w.conv_width,
-                            w.bidirectional, seed=0)
+                            w.bidirectional, seed=0, a_heads=1 if w.extra.get("a_heads") else 0,
+                            bc_shared=bool(w.extra.get("bc_shared")))
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -660,6 +676,17 @@ def main():
             roof = dict(bound="hbm", **{k: hbm[k] for k in ("achieved", "peak", "unit", "frac")},
                         traffic=traffic, peak_kind=hbm["peak_kind"],
                         algorithmic_bytes_per_launch=ab, mean_launch_ms=mean_launch_ms, sfu=sfu)
+        elif w.extra.get("a_heads"):
+            # A per head: one exp per (b, d, l); the floor is the FP32 pipe, three
+            # operations per (b, d, l, n), 128 lanes per SM per clock
+            ops = fp32_ops(w)
+            fp_peak = N_SM * FP32_LANES_PER_SM * sm_mhz * 1e6
+            fp_ach = ops / (mean_launch_ms * 1e-3)
+            roof = dict(bound="alu", achieved=fp_ach / 1e12, peak=fp_peak / 1e12, unit="Tops/s",
+                        frac=fp_ach / fp_peak, traffic=traffic,
+                        peak_kind=(f"{N_SM} SMs x {FP32_LANES_PER_SM} FP32 lanes x {sm_mhz:.0f} MHz "
+                                   "(sampled SM clock)"),
+                        fp32_ops_per_launch=ops, mean_launch_ms=mean_launch_ms, hbm=hbm, sfu=sfu)
         else:
             # one exp per (b, d, l, n) is the binding roof at d_state 16; HBM alongside
             roof = dict(bound="alu", **{k: sfu[k] for k in ("achieved", "peak", "unit", "frac")},

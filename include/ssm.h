@@ -67,8 +67,9 @@ extern "C" {
 #define SSM_API
 #endif
 
-#define SSM_ABI_VERSION 2
-#define SSM_MAX_DSTATE 16
+#define SSM_ABI_VERSION 3
+#define SSM_MAX_DSTATE 16        /* decode (ssm_selective_state_update) */
+#define SSM_MAX_SCAN_DSTATE 128  /* scan (ssm_selective_scan_fwd) */
 #define SSM_MAX_CONV_WIDTH 4
 
 /* A cudaStream_t value, passed through untouched. */
@@ -115,12 +116,13 @@ SSM_API ssm_status_t ssm_causal_conv1d_fwd(const void* x, const float* w, const 
 typedef struct {
     ssm_dtype_t dtype;        /* element type of u, delta, z, B, C, out */
     int64_t batch, dim, seqlen;
-    int64_t dstate;           /* 1..SSM_MAX_DSTATE */
+    int64_t dstate;           /* 1..SSM_MAX_SCAN_DSTATE */
     const void* u;            /* (batch, dim, seqlen); the pre-conv x when conv_weight != NULL */
     const void* delta;        /* (batch, dim, seqlen): raw dt */
-    const float* A;           /* (dim, dstate), normally negative (A = -exp(A_log)) */
-    const void* B;            /* (batch, dstate, seqlen) */
-    const void* C;            /* (batch, dstate, seqlen) */
+    const float* A;           /* (dim, dstate), normally negative (A = -exp(A_log)); with
+                                 a_heads > 0: (a_heads) */
+    const void* B;            /* (batch, dstate, seqlen); with bc_shared: fp32 (dim, dstate) */
+    const void* C;            /* (batch, dstate, seqlen); with bc_shared: fp32 (dim, dstate) */
     const float* D;           /* (dim) skip weight, or NULL (no skip term) */
     const void* z;            /* (batch, dim, seqlen) gate input, or NULL (no gate) */
     const float* delta_bias;  /* (dim) or NULL (zero) */
@@ -129,7 +131,7 @@ typedef struct {
     const float* conv_weight; /* (dim, conv_width) or NULL; non-NULL fuses conv + SiLU on u */
     const float* conv_bias;   /* (dim) or NULL */
     int32_t conv_width;       /* 1..SSM_MAX_CONV_WIDTH when conv_weight != NULL */
-    const float* A_rev;       /* non-NULL selects the bidirectional sum: (dim, dstate) */
+    const float* A_rev;       /* non-NULL selects the bidirectional sum: shaped as A */
     const float* D_rev;       /* (dim) or NULL: skip weight of the reverse direction */
     const float* delta_bias_rev; /* (dim) or NULL: dt bias of the reverse direction */
     void* out;                /* (batch, dim, seqlen) in dtype; must not overlap inputs */
@@ -173,6 +175,19 @@ typedef struct {
      * TMA; otherwise by plain loads. */
     int32_t channel_last;
     int64_t stride_u, stride_delta, stride_z, stride_out, stride_B, stride_C;
+    /* ABI 3. A as one scalar per head (Mamba-2's restriction of the diagonal A,
+     * paperlayer.ai summary of arXiv 2603.09555, §3 Method, "State-space duality"):
+     * a_heads > 0 (dividing dim) makes A and A_rev (a_heads) fp32, head h owning the
+     * dim / a_heads consecutive channels from h * dim / a_heads; every state of those
+     * channels decays by exp(delta * A[h]), one exp per (channel, step). 0: A is
+     * (dim, dstate). */
+    int32_t a_heads;
+    /* Time-invariant B and C (the "variable or shared" B/C dispatch axis, pyshine.com
+     * tour, CUDA-core paragraph): bc_shared = 1 makes B and C fp32 (dim, dstate), the
+     * same at every position (stride_B / stride_C are then ignored); 0: input-dependent
+     * as above. Neither a_heads nor bc_shared combines with seq_starts
+     * (SSM_ERR_UNSUPPORTED); bad values give SSM_ERR_BAD_SHAPE. */
+    int32_t bc_shared;
 } ssm_scan_args_t;
 
 /* Bytes of device workspace the call with these arguments needs (0 if none).

@@ -72,6 +72,15 @@ def _position_stride(t, name):
     return t.stride(1)
 
 
+def _dstate(A, B, channel_last):
+    """d_state: from A (dim, dstate), or, with A given per head, from B."""
+    if A.dim() == 2:
+        return A.shape[1]
+    if B.dim() == 2:                      # time-invariant (dim, dstate)
+        return B.shape[1]
+    return B.shape[2] if channel_last else B.shape[1]
+
+
 def _view_ptr(t):
     return None if t is None or not t.numel() else t.data_ptr()
 
@@ -86,12 +95,20 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, con
         a.channel_last = 1
         a.stride_u, a.stride_delta = _position_stride(u, "u"), _position_stride(delta, "delta")
         a.stride_z, a.stride_out = _position_stride(z, "z"), _position_stride(out, "out")
-        a.stride_B, a.stride_C = _position_stride(B, "B"), _position_stride(C, "C")
-        a.u, a.delta, a.B, a.C, a.z = (_view_ptr(t) for t in (u, delta, B, C, z))
+        if B.dim() == 3:
+            a.stride_B, a.stride_C = _position_stride(B, "B"), _position_stride(C, "C")
+        a.u, a.delta, a.z = (_view_ptr(t) for t in (u, delta, z))
     else:
         batch, dim, seqlen = u.shape
-        a.u, a.delta, a.B, a.C, a.z = _ptr(u), _ptr(delta), _ptr(B), _ptr(C), _ptr(z)
-    a.batch, a.dim, a.seqlen, a.dstate = batch, dim, seqlen, A.shape[1]
+        a.u, a.delta, a.z = _ptr(u), _ptr(delta), _ptr(z)
+    shared = B.dim() == 2                 # time-invariant B, C: fp32 (dim, dstate)
+    if shared:
+        a.B, a.C, a.bc_shared = _fp32(B, "B"), _fp32(C, "C"), 1
+    else:
+        a.B, a.C = (_view_ptr(B), _view_ptr(C)) if channel_last else (_ptr(B), _ptr(C))
+    a.batch, a.dim, a.seqlen = batch, dim, seqlen
+    a.dstate = _dstate(A, B, channel_last)
+    a.a_heads = A.shape[0] if A.dim() == 1 else 0
     a.A, a.D, a.delta_bias = _fp32(A, "A"), _fp32(D, "D"), _fp32(delta_bias, "delta_bias")
     a.delta_softplus, a.reverse = int(bool(delta_softplus)), int(bool(reverse))
     a.conv_weight, a.conv_bias = _fp32(conv_weight, "conv_weight"), _fp32(conv_bias, "conv_bias")
@@ -105,8 +122,10 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, reverse, con
 
 
 def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num_chunks=0,
-                                      reverse=False, seq_starts=None, channel_last=False):
-    """Workspace bytes ssm_selective_scan_fwd needs for these shapes (host-only query)."""
+                                      reverse=False, seq_starts=None, channel_last=False,
+                                      dstate=None, bc_shared=False):
+    """Workspace bytes ssm_selective_scan_fwd needs for these shapes (host-only query).
+    With A given per head (a 1-D tensor), ``dstate`` must be given."""
     lib = _abi.load()
     a = ScanArgs()
     a.dtype = _dtype_code(u)
@@ -115,7 +134,13 @@ def ssm_selective_scan_workspace_size(u, A, *, conv_weight=None, A_rev=None, num
         a.channel_last = 1
     else:
         a.batch, a.dim, a.seqlen = u.shape
-    a.dstate = A.shape[1]
+    if A.dim() == 1:
+        if dstate is None:
+            raise ValueError("A given per head: pass dstate")
+        a.dstate, a.a_heads = int(dstate), A.shape[0]
+    else:
+        a.dstate = A.shape[1]
+    a.bc_shared = int(bool(bc_shared))
     a.reverse = int(bool(reverse))
     a.A_rev = 1 if A_rev is not None else None
     a.conv_weight = 1 if conv_weight is not None else None
@@ -136,8 +161,10 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                            conv_history=None, conv_state_out=None, return_conv_state=False,
                            seq_starts=None, channel_last=False):
     """Selective-scan forward (see include/ssm.h). Layouts: u, delta, z (batch, dim, seqlen);
-    B, C (batch, dstate, seqlen); A (dim, dstate) fp32. With ``conv_weight`` (dim, width), ``u``
-    is the pre-conv x. With ``A_rev`` the result is the bidirectional sum.
+    B, C (batch, dstate, seqlen), or fp32 (dim, dstate) for time-invariant B/C; A (dim,
+    dstate) fp32, or (nheads,) for one scalar per head (d_state then comes from B). With
+    ``conv_weight`` (dim, width), ``u`` is the pre-conv x. With ``A_rev`` (shaped as A) the
+    result is the bidirectional sum.
 
     ``final_state`` / ``final_state_rev`` may be given as preallocated fp32 outputs
     (batch, dim, dstate); they are written whenever given. A forward scan continues a
@@ -163,7 +190,7 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     rows = nseq if seq_starts is not None else u.shape[0]
     dim = u.shape[2] if channel_last else u.shape[1]
     if return_final_state:
-        shp = (rows, dim, A.shape[1])
+        shp = (rows, dim, _dstate(A, B, channel_last))
         if fs is None:
             fs = torch.empty(shp, dtype=torch.float32, device=u.device)
         if A_rev is not None and fsr is None:

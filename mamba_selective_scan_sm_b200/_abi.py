@@ -22,7 +22,7 @@ EXPORTS = (
     "ssm_device_error", "ssm_selective_scan_fwd_noalloc", "ssm_wait_selftest",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
-ABI_VERSION = 2            # SSM_ABI_VERSION of include/ssm.h this mirror follows
+ABI_VERSION = 3            # SSM_ABI_VERSION of include/ssm.h this mirror follows
 
 _P = ctypes.c_void_p
 _FP = ctypes.POINTER(ctypes.c_float)
@@ -46,6 +46,7 @@ class ScanArgs(ctypes.Structure):
         ("seq_starts", _P), ("num_seqs", _I32),
         ("channel_last", _I32), ("stride_u", _I64), ("stride_delta", _I64), ("stride_z", _I64),
         ("stride_out", _I64), ("stride_B", _I64), ("stride_C", _I64),
+        ("a_heads", _I32), ("bc_shared", _I32),
     ]
 
 

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libssm_b200.so")
 SOURCES = ["kernels.cu", "scan_bf16.cu", "scan_f32.cu", "scan_bf16_ext.cu", "scan_f32_ext.cu",
-           "ssm_api.cu", "noalloc.cu"]
+           "scan_bf16_m2.cu", "scan_f32_m2.cu", "ssm_api.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -1,7 +1,8 @@
 // Device code of the library: the conv, decode and self-test kernels, the choice of
-// scan variant and the dispatch to the scan units (scan_bf16.cu, scan_f32.cu and, for
-// packed sequences and channel-last activations, scan_bf16_ext.cu, scan_f32_ext.cu),
-// which hold the scan kernels' instantiations and compile in parallel with this one.
+// scan variant and the dispatch to the scan units (scan_bf16.cu, scan_f32.cu; for
+// packed sequences and channel-last activations scan_bf16_ext.cu, scan_f32_ext.cu; for
+// A per head and time-invariant B/C scan_bf16_m2.cu, scan_f32_m2.cu), which hold the
+// scan kernels' instantiations and compile in parallel with this one.
 #define SSM_ERROR_WORD g_error_main
 #include "conv_kernel.cuh"
 #include "decode_kernel.cuh"
@@ -34,7 +35,7 @@ cudaError_t launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t st) {
 }  // namespace
 
 bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
-#define X(NP_, S_, KC_, SW_, EXT_)                                          \
+#define X(NP_, S_, KC_, SW_, EXT_, M2_)                                     \
     if (np == NP_ && s == S_ && kc == KC_ && sw == SW_) {                   \
         *v = es == 2 ? variant_of<__nv_bfloat16, NP_, S_, KC_, SW_>()       \
                      : variant_of<float, NP_, S_, KC_, SW_>();              \
@@ -45,8 +46,13 @@ bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
     return false;
 }
 
-cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, bool vl, bool cl,
+cudaError_t launch_scan(const ScanVariant& v, bool tma, bool sum, bool vl, bool cl, int feat,
                         const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
+    if (feat) {
+        if (vl) return cudaErrorInvalidValue;
+        return v.elem_size == 2 ? launch_scan_bf16_m2(v, tma, sum, cl, feat, maps, p, grid, st)
+                                : launch_scan_f32_m2(v, tma, sum, cl, feat, maps, p, grid, st);
+    }
     if (vl || cl)
         return v.elem_size == 2 ? launch_scan_bf16_ext(v, tma, sum, vl, cl, maps, p, grid, st)
                                 : launch_scan_f32_ext(v, tma, sum, vl, cl, maps, p, grid, st);
@@ -140,14 +146,16 @@ cudaError_t take_error_main(int* code, cudaStream_t st) {
 }
 
 cudaError_t read_device_error(int* code, cudaStream_t st) {
-    int w[5] = {0, 0, 0, 0, 0};
+    int w[7] = {0, 0, 0, 0, 0, 0, 0};
     cudaError_t e = take_error_main(&w[0], st);
     if (e == cudaSuccess) e = take_error_scan_bf16(&w[1], st);
     if (e == cudaSuccess) e = take_error_scan_f32(&w[2], st);
     if (e == cudaSuccess) e = take_error_scan_bf16_ext(&w[3], st);
     if (e == cudaSuccess) e = take_error_scan_f32_ext(&w[4], st);
+    if (e == cudaSuccess) e = take_error_scan_bf16_m2(&w[5], st);
+    if (e == cudaSuccess) e = take_error_scan_f32_m2(&w[6], st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    *code = w[0] | w[1] | w[2] | w[3] | w[4];
+    *code = w[0] | w[1] | w[2] | w[3] | w[4] | w[5] | w[6];
     return e;
 }
 

@@ -25,9 +25,10 @@ struct ScanVariant {
 // Returns false if (elem_size, np, s, kc, sw) has no compiled kernel.
 bool scan_variant(int elem_size, int np, int s, int kc, int sw, ScanVariant* v);
 
+// feat: bit 0 A as one scalar per head, bit 1 time-invariant B/C (not with packed)
 cudaError_t launch_scan(const ScanVariant& v, bool use_tma, bool summary, bool packed,
-                        bool channel_last, const ScanMaps& maps, const ScanParams& p, dim3 grid,
-                        cudaStream_t stream);
+                        bool channel_last, int feat, const ScanMaps& maps, const ScanParams& p,
+                        dim3 grid, cudaStream_t stream);
 
 cudaError_t launch_conv(int elem_size, bool vec, const ConvParams& p, cudaStream_t stream);
 

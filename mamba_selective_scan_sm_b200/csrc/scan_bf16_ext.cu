@@ -9,7 +9,7 @@ namespace ssm {
 cudaError_t launch_scan_bf16_ext(const ScanVariant& v, bool tma, bool sum, bool vl, bool cl,
                              const ScanMaps& maps, const ScanParams& p, dim3 grid,
                              cudaStream_t st) {
-#define X(NP_, S_, KC_, SW_, EXT_)                                                          \
+#define X(NP_, S_, KC_, SW_, EXT_, M2_)                                                       \
     if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                            \
         return launch_ext<__nv_bfloat16, NP_, S_, KC_, SW_, EXT_>(tma, sum, vl, cl, maps, p, grid, st);
     SSM_SCAN_VARIANTS(X)

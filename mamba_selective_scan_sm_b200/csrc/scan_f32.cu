@@ -8,7 +8,7 @@ namespace ssm {
 
 cudaError_t launch_scan_f32(const ScanVariant& v, bool tma, bool sum, const ScanMaps& maps,
                              const ScanParams& p, dim3 grid, cudaStream_t st) {
-#define X(NP_, S_, KC_, SW_, EXT_)                                                          \
+#define X(NP_, S_, KC_, SW_, EXT_, M2_)                                                       \
     if (v.np == NP_ && v.s == S_ && v.kc == KC_ && v.sw == SW_)                            \
         return launch_v<float, NP_, S_, KC_, SW_, false, false>(tma, sum, maps, p, grid, st);
     SSM_SCAN_VARIANTS(X)

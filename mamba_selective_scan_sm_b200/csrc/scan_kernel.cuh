@@ -71,8 +71,9 @@ struct ScanCfg {
     static constexpr int G = SCAN_THREADS / S * KC;   // channels per CTA
     static constexpr int NT = SCAN_THREADS + kProThreads;   // threads per CTA
     // CTAs per SM the launch bounds ask for: three of 6 warps (96 registers per
-    // thread), three of 4 warps with two channels per lane (168), five of 4 warps (96)
-    static constexpr int MIN_CTAS = SW == 4 ? 3 : (KC == 2 ? 3 : 5);
+    // thread), three of 4 warps with two channels per lane (168), five of 4 warps (96);
+    // two for d_state 64 / 128 (their B/C tiles take up to 113 KB of shared memory)
+    static constexpr int MIN_CTAS = NP * S > 16 ? 2 : (SW == 4 ? 3 : (KC == 2 ? 3 : 5));
     static constexpr int NS = NP * S;            // padded state count
     static constexpr int ES = sizeof(T);
     static constexpr int TT = 64 / ES;           // tile length: 32 (bf16) / 16 (fp32) steps
@@ -112,7 +113,7 @@ struct ScanCfg {
     static_assert(TT % 16 == 0, "tile must hold whole 16-step blocks");
     static_assert(P_PITCH % 16 == 0 && E_PITCH % 16 == 0, "staging rows take 16-byte stores");
     static_assert(BUF_E % 16 == 0 && BUF_BT % 16 == 0 && BUF % 16 == 0, "16-byte aligned parts");
-    static_assert(NS <= 16, "at most 16 states");
+    static_assert(NS <= 128, "at most 128 states");
     static_assert(KC == 1 || KC == 2, "one or two channels per lane");
     static_assert(HALO + TT + 1 <= 64, "the packed-sequence window mask is 64 bits");
 };
@@ -129,7 +130,7 @@ __device__ __forceinline__ int swz(int row, int byte_in_row) {
 // Recurrence state of one lane: NP states, held as fp32 pairs so the four
 // per-state operations (delta*A, delta*u*B, the h update and C.h) issue as packed
 // .f32x2 instructions.
-template <int NP, bool SUMMARY>
+template <int NP, bool SUMMARY, bool SA = false>
 struct LaneState {
     static constexpr int NPR = NP / 2;                   // packed pairs
     static constexpr bool ODD = (NP % 2) != 0;
@@ -178,19 +179,24 @@ struct LaneState {
         float dA1, bu1, c1;
     };
 
-    // dl = delta, du = delta*u of the step; b / cvv: this lane's NP fp32 B and C values.
+    // dl = delta (SA: the step's decay dA itself, the same for every state of a head),
+    // du = delta*u of the step; b / cvv: this lane's NP fp32 B and C values.
     __device__ __forceinline__ In prep(float dl, float du, const float* b, const float* cvv) const {
         In in;
         const uint64_t dd = pk2(dl, dl), uu = pk2(du, du);
 #pragma unroll
         for (int k = 0; k < NPR; ++k) {
-            const uint64_t x = mul2(dd, a2[k]);
-            in.dA[k] = pk2(ex2(lo2(x)), ex2(hi2(x)));
+            if (SA) {
+                in.dA[k] = dd;
+            } else {
+                const uint64_t x = mul2(dd, a2[k]);
+                in.dA[k] = pk2(ex2(lo2(x)), ex2(hi2(x)));
+            }
             in.bu[k] = mul2(uu, pk2(b[2 * k], b[2 * k + 1]));
             if (!SUMMARY) in.cc[k] = pk2(cvv[2 * k], cvv[2 * k + 1]);
         }
         if (ODD) {
-            in.dA1 = ex2(dl * a1);
+            in.dA1 = SA ? dl : ex2(dl * a1);
             in.bu1 = du * b[NP - 1];
             if (!SUMMARY) in.c1 = cvv[NP - 1];
         }
@@ -236,7 +242,7 @@ __device__ __noinline__ void put_conv_history(const ScanParams& p, uint8_t* raw_
 }
 
 template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY, bool VL,
-          bool CL>
+          bool CL, int FEAT>
 __global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
@@ -245,10 +251,18 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     constexpr int G = Cfg::G, NS = Cfg::NS, TT = Cfg::TT, HALO = Cfg::HALO, R = Cfg::R;
     constexpr int ROWB = Cfg::ROWB, SWZ = Cfg::SWZ;
     constexpr int NSTAGE = Cfg::NSTAGE;
+    // FEAT bit 0 (SA): A is one scalar per head; the producers stage the step's decay
+    // exp(delta A_h) in place of delta and the scan warps take no exps. Bit 1 (SB): B and
+    // C are fp32 (dim, dstate), fixed per channel; no B/C tiles, each lane keeps its
+    // channel's NP values of each in registers.
+    constexpr bool SA = (FEAT & 1) != 0, SB = (FEAT & 2) != 0;
+    static_assert(!SB || KC == 1, "time-invariant B/C: one channel per lane");
 
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base, reached by pointer arithmetic on the shared array (not
+    // through an integer cast) so that every pointer derived from it stays in the
+    // shared address space and its loads compile to shared loads, not generic ones
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float* par = reinterpret_cast<float*>(smem + Cfg::OFF_PAR);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* full_raw = bars;                    // [NSTAGE] TMA bytes landed (1 arrival + tx)
@@ -305,7 +319,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         q[8] = q[9] = (ok && p.conv_b) ? p.conv_b[dd] : 0.f;
         q[10] = q[11] = (ok && p.dbias[dir]) ? p.dbias[dir][dd] : 0.f;
         q[12] = q[13] = (ok && p.Dv[dir]) ? p.Dv[dir][dd] : 0.f;
-        q[14] = q[15] = 0.f;
+        q[14] = q[15] = (SA && ok) ? p.A[dir][dd / p.head_dim] * kLog2e : 0.f;   // A_h log2(e)
     }
     __syncthreads();   // barriers initialised and parameters written, for both roles
 
@@ -318,19 +332,23 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const int l0 = tile_l0(f);
             const bool rv = tile_rev(f);
             const uint32_t bytes =
-                2u * NS * ROWB + G * xpitch + G * ROWB + (has_z ? G * ROWB : 0u);
+                (SB ? 0u : 2u * NS * ROWB) + G * xpitch + G * ROWB + (has_z ? G * ROWB : 0u);
             uint64_t* bar = &full_raw[f % NSTAGE];
             mbar_arrive_expect_tx(bar, bytes);
             const int lx = (conv && !rv) ? l0 - HALO : l0;
             if constexpr (CL) {               // maps over (channel, t, batch)
-                tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, 0, l0, b);
-                tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, 0, l0, b);
+                if (!SB) {
+                    tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, 0, l0, b);
+                    tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, 0, l0, b);
+                }
                 tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, d0, lx, b);
                 tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, d0, l0, b);
                 if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, d0, l0, b);
             } else {                          // maps over (t, channel, batch)
-                tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, l0, 0, b);
-                tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, l0, 0, b);
+                if (!SB) {
+                    tma_load_3d(st + Cfg::RAW_B, &maps.B, bar, l0, 0, b);
+                    tma_load_3d(st + Cfg::RAW_C, &maps.C, bar, l0, 0, b);
+                }
                 tma_load_3d(st + Cfg::RAW_X, &maps.x, bar, lx, d0, b);
                 tma_load_3d(st + Cfg::RAW_DT, &maps.dt, bar, l0, d0, b);
                 if (has_z) tma_load_3d(st + Cfg::RAW_Z, &maps.z, bar, l0, d0, b);
@@ -344,7 +362,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const int l0 = tile_l0(f);
             const bool rv = tile_rev(f);
             const int64_t bL = (int64_t)b * L;
-            for (int e = ptid; e < NS * TT; e += kProThreads) {
+            for (int e = ptid; e < (SB ? 0 : NS * TT); e += kProThreads) {
                 const int n = e % NS, row = e / NS, t = l0 + row;
                 const bool ok = n < p.dstate && t >= 0 && t < L;
                 reinterpret_cast<T*>(st + Cfg::RAW_B)[e] =
@@ -381,7 +399,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const bool rv = tile_rev(f);
             const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
             const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
-            for (int e = ptid; e < NS * TT; e += kProThreads) {
+            for (int e = ptid; e < (SB ? 0 : NS * TT); e += kProThreads) {
                 const int n = e / TT, col = e % TT, t = l0 + col;
                 const bool ok = n < p.dstate && t >= 0 && t < L;
                 const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
@@ -450,8 +468,10 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             static_assert(SEG % SUB == 0 && SUB % EPC == 0 && SUB % 2 == 0, "windows of whole chunks");
             // B, C: swizzled [n][t] -> fp32 [t][n] (channel-last: already [t][n], widened
             // only), one 16-byte chunk per thread and pass
-            constexpr int NCH = NS * ROWB / 16;               // chunks per tensor
-            if constexpr (CL) {
+            [[maybe_unused]] constexpr int NCH = NS * ROWB / 16;   // chunks per tensor
+            if constexpr (SB) {
+                // time-invariant B/C: nothing staged per tile
+            } else if constexpr (CL) {
                 for (int e = ptid; e < 2 * NCH; e += kProThreads) {
                     const int ten = e / NCH, ch = e % NCH;
                     const uint4 v[1] = {reinterpret_cast<const uint4*>(
@@ -492,6 +512,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const uint64_t cb2 = pk2(__uint_as_float(qc.x), __uint_as_float(qc.y));
             const uint64_t bias2 = pk2(__uint_as_float(qc.z), __uint_as_float(qc.w));
             const uint64_t D2 = pk2(__uint_as_float(qd.x), __uint_as_float(qd.y));
+            [[maybe_unused]] const float aH = __uint_as_float(qd.z);   // SA: A_h log2(e)
             // P rows hold KC channels side by side: this channel's {delta, delta*u} slot
             uint8_t* prow_base = buf + Cfg::BUF_P + (r / KC) * Cfg::P_PITCH + (r % KC) * 8;
             // packed sequences: the conv of step ti reads no position before its start
@@ -562,7 +583,9 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     }
                     uint64_t dl2 = add2(pk2(DT(i), DT(i + 1)), bias2);
                     if (p.softplus) dl2 = softplus2(dl2);
-                    const float2 dl = upk2(dl2), du = upk2(mul2(dl2, u2));
+                    float2 dl = upk2(dl2);
+                    const float2 du = upk2(mul2(dl2, u2));
+                    if (SA) dl = make_float2(ex2(dl.x * aH), ex2(dl.y * aH));   // the decay
                     if constexpr (KC == 1) {
                         *reinterpret_cast<float4*>(prow + i * 8) = make_float4(dl.x, du.x, dl.y, du.y);
                     } else {
@@ -645,7 +668,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     auto chan_d = [&](int k) { return d0 + lg * KC + k; };                 // channel k of the lane
     auto chan_row = [&](int k) { return (int64_t)b * p.dim + chan_d(k); };  // its (b, d) row
 
-    LaneState<NP, SUMMARY> ls[KC];
+    LaneState<NP, SUMMARY, SA> ls[KC];
     auto load_A = [&](int dir) {
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
@@ -654,12 +677,24 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll
             for (int i = 0; i < NP; ++i) {
                 const int n = j * NP + i;
-                a[i] = (d < p.dim && n < p.dstate) ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e
-                                                   : 0.f;
+                a[i] = (!SA && d < p.dim && n < p.dstate)
+                           ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
             }
             ls[k].set_a(a);
         }
     };
+    // SB: the lane's NP values of its channel's fixed B and C rows, for every step
+    [[maybe_unused]] float sb_b[NP], sb_c[NP];
+    if constexpr (SB) {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+            const int n = j * NP + i;
+            const bool ok = chan_d(0) < p.dim && n < p.dstate;
+            const int64_t o = (int64_t)chan_d(0) * p.dstate + n;
+            sb_b[i] = ok ? static_cast<const float*>(p.Bm)[o] : 0.f;
+            sb_c[i] = ok ? static_cast<const float*>(p.Cm)[o] : 0.f;
+        }
+    }
     // Initial state of this chunk: carry over the summaries of earlier chunks.
     // A caller's initial state (a continued sequence) is the carry into chunk 0.
     auto init_state = [&]() {
@@ -821,8 +856,8 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 }
             }
         };
-        const float* Bl = reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * NP;
-        const float* Cl = reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * NP;
+        [[maybe_unused]] const float* Bl = reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * NP;
+        [[maybe_unused]] const float* Cl = reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * NP;
         // {delta, delta*u} of step tt for the lane's KC channels
         auto load_p = [&](int tt, float2 (&pd)[KC]) {
             if constexpr (KC == 2) {
@@ -835,7 +870,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         };
         // this lane's NP values of B and C at step tt
         auto load_bc = [&](int tt, float (&bv)[NP], float (&cv)[NP]) {
-            if constexpr (NP % 4 == 0) {
+            if constexpr (SB) {
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    bv[i] = sb_b[i];
+                    cv[i] = sb_c[i];
+                }
+            } else if constexpr (NP % 4 == 0) {
 #pragma unroll
                 for (int i = 0; i < NP; i += 4) {
                     const float4 b4 = *reinterpret_cast<const float4*>(Bl + tt * NS + i);
@@ -871,7 +912,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 constexpr int KB = SSM_SCAN_BATCH;
 #pragma unroll
                 for (int q0 = 0; q0 < 16; q0 += KB) {
-                    typename LaneState<NP, SUMMARY>::In in[KB][KC];
+                    typename LaneState<NP, SUMMARY, SA>::In in[KB][KC];
 #pragma unroll
                     for (int u = 0; u < KB; ++u) {
                         const int tt = RV ? TT - 1 - (blk * 16 + q0 + u) : blk * 16 + q0 + u;

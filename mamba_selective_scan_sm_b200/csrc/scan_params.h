@@ -43,6 +43,10 @@ struct ScanParams {
     // channel-last activations: element strides between consecutive positions
     int64_t su, sdl, sz, sout, sB, sC, spart;
     int vec_store;          // rows are 16-byte aligned: vector stores allowed
+    // A as one scalar per head (kernels with FEAT bit 0): channels per head; A[dir] is
+    // (dim / head_dim,) and channel d uses A[dir][d / head_dim]
+    int head_dim;
+    // time-invariant B, C (kernels with FEAT bit 1): Bm, Cm are fp32 (dim, dstate)
 };
 
 // The last conv_width inputs of history ++ x per row (the conv state a decode step

@@ -126,9 +126,17 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
     if (a->batch < 0 || a->dim < 0 || a->seqlen < 0)
         return fail(SSM_ERR_BAD_SHAPE, "negative size (batch %lld, dim %lld, seqlen %lld)",
                     (long long)a->batch, (long long)a->dim, (long long)a->seqlen);
-    if (a->dstate < 1 || a->dstate > SSM_MAX_DSTATE)
+    if (a->dstate < 1 || a->dstate > SSM_MAX_SCAN_DSTATE)
         return fail(SSM_ERR_BAD_SHAPE, "dstate %lld outside 1..%d", (long long)a->dstate,
-                    SSM_MAX_DSTATE);
+                    SSM_MAX_SCAN_DSTATE);
+    if (a->a_heads < 0 || (a->a_heads > 0 && a->dim % a->a_heads != 0))
+        return fail(SSM_ERR_BAD_SHAPE, "a_heads %d must be 0 or divide dim %lld", a->a_heads,
+                    (long long)a->dim);
+    if (a->bc_shared != 0 && a->bc_shared != 1)
+        return fail(SSM_ERR_BAD_SHAPE, "bc_shared %d is not 0 or 1", a->bc_shared);
+    if ((a->a_heads > 0 || a->bc_shared) && a->seq_starts)
+        return fail(SSM_ERR_UNSUPPORTED,
+                    "packed sequences need per-state A and input-dependent B, C");
     if (a->seqlen > 0x3fffffffLL || a->dim > 0x3fffffffLL)
         return fail(SSM_ERR_BAD_SHAPE, "seqlen and dim must be below 2^30");
     if (a->batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch %lld > 65535", (long long)a->batch);
@@ -169,9 +177,17 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
     }
 
     const int es = elem_size(a->dtype);
-    const int ns = a->dstate <= 4 ? 4 : a->dstate <= 8 ? 8 : 16;
+    const int ns = a->dstate <= 4    ? 4
+                   : a->dstate <= 8  ? 8
+                   : a->dstate <= 16 ? 16
+                   : a->dstate <= 64 ? 64
+                                     : 128;
     int np = 4, s = 4, kc = 1, sw = 4;
-    if (ns == 16) {
+    if (ns > 16) {
+        // d_state 64 / 128: 16 lanes per channel of 4 / 8 states, 8 channels per CTA
+        s = 16;
+        np = ns / 16;
+    } else if (ns == 16) {
         // Batch rows with enough channels for two 32-channel CTAs per SM: 4 lanes per
         // channel (4 states each) in CTAs of 4 scan warps. Fewer channels: 8 lanes per
         // channel in CTAs of 2 scan warps (8 channels each), for more CTAs and warps.
@@ -182,7 +198,8 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         if (s != 4 && s != 8) s = 4;
         kc = env_int("SSM_CHANNELS_PER_LANE", 1);
         if (kc != 1 && kc != 2) kc = 1;
-        if (a->seq_starts || a->channel_last) kc = 1;   // the splits compiled for those
+        if (a->seq_starts || a->channel_last || a->a_heads > 0 || a->bc_shared)
+            kc = 1;                                     // the splits compiled for those
         np = 16 / s;
         sw = (s == 4) == (kc == 1) ? 4 : 2;
     } else if (ns == 8) {
@@ -277,8 +294,9 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     const int64_t sdl = cl ? (a->stride_delta ? a->stride_delta : a->dim) : 0;
     const int64_t sz = cl ? (a->stride_z ? a->stride_z : a->dim) : 0;
     const int64_t sout = cl ? (a->stride_out ? a->stride_out : a->dim) : 0;
-    const int64_t sB = cl ? (a->stride_B ? a->stride_B : a->dstate) : 0;
-    const int64_t sC = cl ? (a->stride_C ? a->stride_C : a->dstate) : 0;
+    const bool sb = a->bc_shared != 0;            // B, C fp32 (dim, dstate), fixed per channel
+    const int64_t sB = (cl && !sb) ? (a->stride_B ? a->stride_B : a->dstate) : 0;
+    const int64_t sC = (cl && !sb) ? (a->stride_C ? a->stride_C : a->dstate) : 0;
     // bytes each tensor spans: (batch, dim, seqlen) dense, or batch*seqlen positions at
     // their stride, the last one `width` elements long
     const int64_t npos = a->batch * a->seqlen;
@@ -289,7 +307,9 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     const size_t bc = (size_t)a->batch * a->dstate * a->seqlen * es;
     const size_t act_u = cl ? span(su, a->dim) : act, act_dl = cl ? span(sdl, a->dim) : act;
     const size_t act_z = cl ? span(sz, a->dim) : act, act_out = cl ? span(sout, a->dim) : act;
-    const size_t bc_B = cl ? span(sB, a->dstate) : bc, bc_C = cl ? span(sC, a->dstate) : bc;
+    const size_t bc_fixed = (size_t)a->dim * a->dstate * sizeof(float);
+    const size_t bc_B = sb ? bc_fixed : cl ? span(sB, a->dstate) : bc;
+    const size_t bc_C = sb ? bc_fixed : cl ? span(sC, a->dstate) : bc;
     const bool empty = rows == 0 || a->seqlen == 0;
 
     if (!empty) {
@@ -302,7 +322,8 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     // element alignment
     struct { const void* p; size_t al; const char* n; } al[] = {
         {a->u, (size_t)es, "u"}, {a->delta, (size_t)es, "delta"}, {a->z, (size_t)es, "z"},
-        {a->B, (size_t)es, "B"}, {a->C, (size_t)es, "C"}, {a->out, (size_t)es, "out"},
+        {a->B, sb ? 4 : (size_t)es, "B"}, {a->C, sb ? 4 : (size_t)es, "C"},
+        {a->out, (size_t)es, "out"},
         {a->A, 4, "A"}, {a->D, 4, "D"}, {a->delta_bias, 4, "delta_bias"},
         {a->conv_weight, 4, "conv_weight"}, {a->conv_bias, 4, "conv_bias"},
         {a->A_rev, 4, "A_rev"}, {a->D_rev, 4, "D_rev"}, {a->delta_bias_rev, 4, "delta_bias_rev"},
@@ -414,6 +435,8 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     p.sout = sout;
     p.sB = sB;
     p.sC = sC;
+    p.head_dim = a->a_heads > 0 ? (int)(a->dim / a->a_heads) : 0;
+    const int feat = (a->a_heads > 0 ? 1 : 0) | (sb ? 2 : 0);
     if (bidir) {
         // the forward sweep's fp32 partial y: in `out` itself when fp32 (same layout and
         // stride), else in the workspace (dense, the activations' layout)
@@ -428,10 +451,12 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     // TMA needs 16-byte aligned bases and strides of a multiple of 16 bytes (and, in
     // channel-last, B/C rows of at least 16 bytes)
     const int ns_pad = pl.v.np * pl.v.s;
-    const bool strides16 = cl ? ((su | sdl | sz | sB | sC) * es) % 16 == 0 && ns_pad * es >= 16
+    const bool strides16 = cl ? ((su | sdl | sz | sB | sC) * es) % 16 == 0 &&
+                                    (sb || ns_pad * es >= 16)
                               : row16;
-    bool tma = strides16 && aligned(a->u, 16) && aligned(a->delta, 16) && aligned(a->B, 16) &&
-               aligned(a->C, 16) && (!a->z || aligned(a->z, 16)) && env_int("SSM_NO_TMA", 0) == 0;
+    bool tma = strides16 && aligned(a->u, 16) && aligned(a->delta, 16) &&
+               (sb || (aligned(a->B, 16) && aligned(a->C, 16))) && (!a->z || aligned(a->z, 16)) &&
+               env_int("SSM_NO_TMA", 0) == 0;
     ssm::ScanMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (tma) {
@@ -453,25 +478,26 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
             tma = map(&maps.x, a->u, D, su, v.channels, xbox) &&
                   map(&maps.dt, a->delta, D, sdl, v.channels, v.tile) &&
                   (!a->z || map(&maps.z, a->z, D, sz, v.channels, v.tile)) &&
-                  map(&maps.B, a->B, N, sB, ns_pad, v.tile) &&
-                  map(&maps.C, a->C, N, sC, ns_pad, v.tile);
+                  (sb || (map(&maps.B, a->B, N, sB, ns_pad, v.tile) &&
+                          map(&maps.C, a->C, N, sC, ns_pad, v.tile)));
         } else {
             tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
                   encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
                   (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, none)) &&
-                  encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
-                  encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc);
+                  (sb || (encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
+                          encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc)));
         }
     }
 
     const unsigned gx = (unsigned)((a->dim + pl.v.channels - 1) / pl.v.channels);
     cudaError_t e;
     if (pl.nchunks > 1) {
-        e = ssm::launch_scan(pl.v, tma, true, packed, cl, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks - 1),
-                             s);
+        e = ssm::launch_scan(pl.v, tma, true, packed, cl, feat, maps, p,
+                             dim3(gx, (unsigned)a->batch, pl.nchunks - 1), s);
         if (e != cudaSuccess) return cuda_fail(e, "summary pass launch");
     }
-    e = ssm::launch_scan(pl.v, tma, false, packed, cl, maps, p, dim3(gx, (unsigned)a->batch, pl.nchunks), s);
+    e = ssm::launch_scan(pl.v, tma, false, packed, cl, feat, maps, p,
+                         dim3(gx, (unsigned)a->batch, pl.nchunks), s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     if (ssm_status_t t = conv_tail(); t != SSM_OK) return t;
     return ok();

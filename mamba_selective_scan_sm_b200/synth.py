@@ -14,7 +14,8 @@ describes it, section "Why You Need This": dt bias placed so that softplus of
 it lies in [dt_min, dt_max]; A from the S4D-real initialisation, kept in fp32):
 
 * u (or the pre-conv x), z, B, C ~ N(0, 1)
-* A[d, n] = -(n + 1)
+* A[d, n] = -(n + 1); A given per head (Mamba-2 style): A[h] = -U(1, 16)
+* time-invariant B, C: fp32 (dim, dstate) ~ N(0, 1)
 * D ~ N(0, 1)
 * dt_bias[d] = log(expm1(y)), y = exp(U(ln 1e-3, ln 0.1)) per channel
 * dt_raw ~ N(0, 0.5**2)
@@ -32,7 +33,8 @@ TID = {
     "u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "D": 6, "delta_bias": 7,
     "conv_w": 8, "D_rev": 9, "delta_bias_rev": 10, "state": 11, "conv_state": 12,
     "dec_x": 13, "dec_dt": 14, "dec_z": 15, "dec_B": 16, "dec_C": 17,
-    "A_rev": 18, "lengths": 19,
+    "A_rev": 18, "lengths": 19, "A_heads": 20, "A_heads_rev": 21, "B_fixed": 22,
+    "C_fixed": 23,
 }
 
 
@@ -66,6 +68,11 @@ def normal(seed: int, role: str, shape, std: float = 1.0) -> np.ndarray:
 
 def s4d_real_A(dim: int, dstate: int) -> np.ndarray:
     return np.tile(-np.arange(1, dstate + 1, dtype=np.float32), (dim, 1))
+
+
+def heads_A(seed: int, role: str, nheads: int) -> np.ndarray:
+    """One negative scalar per head, -U(1, 16)."""
+    return (-rng(seed, TID[role]).uniform(1.0, 16.0, size=nheads)).astype(np.float32)
 
 
 def dt_bias(seed: int, role: str, dim: int, dt_min=1e-3, dt_max=0.1) -> np.ndarray:
@@ -110,6 +117,9 @@ WORKLOADS = {
                         "x, z halves of one (B, L, 2D) in_proj output; B, C columns of one "
                         "(B, L, 48 + 2N) x_proj output", 8, 1536, 2048, 16, "bf16", conv_width=4,
                         extra={"channel_last": True, "dt_rank": 48}),
+    "heads128": Workload("Mamba-2-130M-shaped scan B8 L2048 D1536 (24 heads x 64) N128 bf16 + "
+                         "conv4: A one scalar per head", 8, 1536, 2048, 128, "bf16", conv_width=4,
+                         extra={"a_heads": 24}),
     "varlen": Workload("packed sequences B1 D1536 L32768 N16 bf16 + conv4, lengths "
                        "log-uniform in [64, 4096]", 1, 1536, 32768, 16, "bf16", conv_width=4,
                        final_state=True, extra={"packed": (64, 4096)}),
@@ -132,11 +142,13 @@ def _act(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def scan_inputs(batch: int, dim: int, seqlen: int, dstate: int = 16, dtype: str = "f32",
-                conv_width: int = 0, bidirectional: bool = False, seed: int = 0) -> dict:
+                conv_width: int = 0, bidirectional: bool = False, seed: int = 0,
+                a_heads: int = 0, bc_shared: bool = False) -> dict:
     """All inputs of one scan call as fp32 numpy arrays (activations bf16-rounded if bf16).
 
-    Layouts: u, delta, z (batch, dim, seqlen); B, C (batch, dstate, seqlen);
-    A (dim, dstate); D, delta_bias (dim); conv_w (dim, conv_width); conv_b (dim).
+    Layouts: u, delta, z (batch, dim, seqlen); B, C (batch, dstate, seqlen), or fp32
+    (dim, dstate) with ``bc_shared``; A (dim, dstate), or (a_heads,) with ``a_heads``;
+    D, delta_bias (dim); conv_w (dim, conv_width); conv_b (dim).
     """
     shp = (batch, dim, seqlen)
     out = {
@@ -156,6 +168,13 @@ def scan_inputs(batch: int, dim: int, seqlen: int, dstate: int = 16, dtype: str 
         out["A_rev"] = s4d_real_A(dim, dstate)
         out["D_rev"] = normal(seed, "D_rev", (dim,))
         out["delta_bias_rev"] = dt_bias(seed, "delta_bias_rev", dim)
+    if a_heads:
+        out["A"] = heads_A(seed, "A_heads", a_heads)
+        if bidirectional:
+            out["A_rev"] = heads_A(seed, "A_heads_rev", a_heads)
+    if bc_shared:
+        out["B"] = normal(seed, "B_fixed", (dim, dstate))
+        out["C"] = normal(seed, "C_fixed", (dim, dstate))
     return out
 
 

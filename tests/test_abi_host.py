@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 2
+    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 3
     for code, name in _abi.STATUS.items():
         assert lib.ssm_status_string(code)
     assert lib.ssm_status_string(999) == b"unknown status"
@@ -71,7 +71,10 @@ def _scan(lib, a):
 @pytest.mark.parametrize("field,value,status", [
     ("dtype", 7, "SSM_ERR_BAD_DTYPE"),
     ("dstate", 0, "SSM_ERR_BAD_SHAPE"),
-    ("dstate", 17, "SSM_ERR_BAD_SHAPE"),
+    ("dstate", 129, "SSM_ERR_BAD_SHAPE"),
+    ("a_heads", 5, "SSM_ERR_BAD_SHAPE"),          # does not divide dim 64
+    ("a_heads", -1, "SSM_ERR_BAD_SHAPE"),
+    ("bc_shared", 2, "SSM_ERR_BAD_SHAPE"),
     ("seqlen", -1, "SSM_ERR_BAD_SHAPE"),
     ("batch", 70000, "SSM_ERR_UNSUPPORTED"),
     ("num_chunks", -2, "SSM_ERR_BAD_SHAPE"),
@@ -120,6 +123,10 @@ CONV = dict(conv_weight=FAKE + (1 << 30), conv_width=4)
      "SSM_ERR_UNSUPPORTED"),
     (dict(seq_starts=FAKE + (1 << 29), num_seqs=0, batch=1), "SSM_ERR_BAD_SHAPE"),
     (dict(seq_starts=FAKE + (1 << 29) + 2, num_seqs=3, batch=1), "SSM_ERR_MISALIGNED"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3, batch=1, a_heads=4), "SSM_ERR_UNSUPPORTED"),
+    (dict(seq_starts=FAKE + (1 << 29), num_seqs=3, batch=1, bc_shared=1), "SSM_ERR_UNSUPPORTED"),
+    # time-invariant B, C are fp32: 4-byte alignment even for bf16 activations
+    (dict(bc_shared=1, B=FAKE + 3 * (1 << 24) + 2), "SSM_ERR_MISALIGNED"),
 ])
 def test_scan_continuation_arguments(lib, kw, status):
     """initial_state / conv_history / conv_state_out: forward scans, a fused conv for the
@@ -173,6 +180,10 @@ def test_workspace_size_query(lib):
     a = _args(A_rev=FAKE + (1 << 30), dtype=0)        # fp32 bidirectional: out holds it
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 0
+    # d_state 100 runs in the 128-state split: the carry holds 128 (P, S) pairs per row
+    a = _args(num_chunks=4, batch=1, dim=64, seqlen=4096, dstate=100, a_heads=8)
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 3 * 1 * 64 * 128 * 8
 
 
 def test_scan_workspace_too_small(lib):
