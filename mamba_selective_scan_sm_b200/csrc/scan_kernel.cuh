@@ -667,6 +667,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     const int j = tid % S;          // state group of this lane
     auto chan_d = [&](int k) { return d0 + lg * KC + k; };                 // channel k of the lane
     auto chan_row = [&](int k) { return (int64_t)b * p.dim + chan_d(k); };  // its (b, d) row
+    // The state in slot i of this lane. With NP a multiple of 4 the lanes interleave in
+    // groups of 4 states, so that a quarter warp's 16-byte B/C loads are contiguous
+    // (NP = 8 with lanes owning 8 consecutive states would put lanes j and j + 4 on the
+    // same banks); otherwise lane j owns states j*NP .. j*NP + NP - 1.
+    auto state_n = [&](int i) {
+        return NP % 4 == 0 ? (i >> 2) * (4 * S) + 4 * j + (i & 3) : j * NP + i;
+    };
 
     LaneState<NP, SUMMARY, SA> ls[KC];
     auto load_A = [&](int dir) {
@@ -676,7 +683,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             float a[NP];
 #pragma unroll
             for (int i = 0; i < NP; ++i) {
-                const int n = j * NP + i;
+                const int n = state_n(i);
                 a[i] = (!SA && d < p.dim && n < p.dstate)
                            ? p.A[dir][(int64_t)d * p.dstate + n] * kLog2e : 0.f;
             }
@@ -688,7 +695,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     if constexpr (SB) {
 #pragma unroll
         for (int i = 0; i < NP; ++i) {
-            const int n = j * NP + i;
+            const int n = state_n(i);
             const bool ok = chan_d(0) < p.dim && n < p.dstate;
             const int64_t o = (int64_t)chan_d(0) * p.dstate + n;
             sb_b[i] = ok ? static_cast<const float*>(p.Bm)[o] : 0.f;
@@ -705,7 +712,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 float hv[NP];
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    const int n = j * NP + i;
+                    const int n = state_n(i);
                     hv[i] = (p.h0 && n < p.dstate) ? p.h0[chan_row(k) * p.dstate + n] : 0.f;
                 }
                 const int64_t stride = (int64_t)p.batch * p.dim * NS;
@@ -851,13 +858,17 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 float* fs = p.final_state[0] + ((int64_t)q * p.dim + chan_d(k)) * p.dstate;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    const int n = j * NP + i;
+                    const int n = state_n(i);
                     if (n < p.dstate) fs[n] = ls[k].get(i);
                 }
             }
         };
-        [[maybe_unused]] const float* Bl = reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * NP;
-        [[maybe_unused]] const float* Cl = reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * NP;
+        // this lane's first B/C value of a step (its slot 0; see state_n)
+        constexpr int kLaneOff = NP % 4 == 0 ? 4 : NP;
+        [[maybe_unused]] const float* Bl =
+            reinterpret_cast<const float*>(buf + Cfg::BUF_BT) + j * kLaneOff;
+        [[maybe_unused]] const float* Cl =
+            reinterpret_cast<const float*>(buf + Cfg::BUF_CT) + j * kLaneOff;
         // {delta, delta*u} of step tt for the lane's KC channels
         auto load_p = [&](int tt, float2 (&pd)[KC]) {
             if constexpr (KC == 2) {
@@ -879,10 +890,11 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             } else if constexpr (NP % 4 == 0) {
 #pragma unroll
                 for (int i = 0; i < NP; i += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(Bl + tt * NS + i);
+                    const int o = tt * NS + (i >> 2) * (4 * S);      // slots i .. i + 3
+                    const float4 b4 = *reinterpret_cast<const float4*>(Bl + o);
                     bv[i] = b4.x; bv[i + 1] = b4.y; bv[i + 2] = b4.z; bv[i + 3] = b4.w;
                     if (!SUMMARY) {
-                        const float4 c4 = *reinterpret_cast<const float4*>(Cl + tt * NS + i);
+                        const float4 c4 = *reinterpret_cast<const float4*>(Cl + o);
                         cv[i] = c4.x; cv[i + 1] = c4.y; cv[i + 2] = c4.z; cv[i + 3] = c4.w;
                     }
                 }
@@ -982,7 +994,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 float* fs = p.final_state[dir] + row * p.dstate;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    const int n = j * NP + i;
+                    const int n = state_n(i);
                     if (n < p.dstate) fs[n] = ls[k].get(i);
                 }
             }

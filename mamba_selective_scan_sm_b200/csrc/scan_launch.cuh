@@ -42,11 +42,16 @@ cudaError_t launch_ext(bool tma, bool sum, bool vl, bool cl, const ScanMaps& map
     return cudaErrorInvalidValue;
 }
 
-// A per head / time-invariant B/C (feat 1..3), either layout: only splits marked M2
-template <typename T, int NP, int S, int KC, int SW, bool M2>
+// A per head / time-invariant B/C (feat 1..3), either layout: splits marked M2 = 1; A per
+// head only (feat 1): splits marked M2 = 2
+template <typename T, int NP, int S, int KC, int SW, int M2>
 cudaError_t launch_m2(bool tma, bool sum, bool cl, int feat, const ScanMaps& maps,
                       const ScanParams& p, dim3 grid, cudaStream_t st) {
-    if constexpr (M2) {
+    if constexpr (M2 == 2) {
+        if (feat == 1)
+            return cl ? launch_v<T, NP, S, KC, SW, false, true, 1>(tma, sum, maps, p, grid, st)
+                      : launch_v<T, NP, S, KC, SW, false, false, 1>(tma, sum, maps, p, grid, st);
+    } else if constexpr (M2 == 1) {
         switch (feat | (cl ? 4 : 0)) {
             case 1: return launch_v<T, NP, S, KC, SW, false, false, 1>(tma, sum, maps, p, grid, st);
             case 2: return launch_v<T, NP, S, KC, SW, false, false, 2>(tma, sum, maps, p, grid, st);

@@ -6,9 +6,10 @@
 namespace ssm {
 
 // (states per lane, lanes per channel, channels per lane, scan warps per CTA, EXT, M2):
-// EXT splits also have packed-sequence and channel-last kernels; M2 splits also have
-// kernels for A as one scalar per head and for time-invariant B/C. 16 lanes of 4 or 8
-// states cover d_state 64 and 128.
+// EXT splits also have packed-sequence and channel-last kernels; M2 = 1 splits also have
+// kernels for A as one scalar per head and for time-invariant B/C, M2 = 2 splits for A
+// per head only. 16 lanes of 4 or 8 states cover d_state 64 and 128; with A per head
+// two channels per lane share each B/C load.
 #define SSM_SCAN_VARIANTS(X) \
     X(4, 4, 1, 4, 1, 1)      \
     X(4, 4, 2, 2, 0, 0)      \
@@ -17,7 +18,9 @@ namespace ssm {
     X(2, 4, 1, 4, 1, 1)      \
     X(1, 4, 1, 4, 1, 1)      \
     X(4, 16, 1, 4, 1, 1)     \
-    X(8, 16, 1, 4, 1, 1)
+    X(8, 16, 1, 4, 1, 1)     \
+    X(4, 16, 2, 4, 0, 2)     \
+    X(8, 16, 2, 4, 0, 2)
 
 // One scan pass with split `v`: one sequence per row in the (batch, dim, seqlen)
 // layout (scan_bf16.cu / scan_f32.cu), packed sequences / channel-last

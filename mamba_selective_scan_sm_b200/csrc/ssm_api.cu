@@ -184,9 +184,13 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
                                      : 128;
     int np = 4, s = 4, kc = 1, sw = 4;
     if (ns > 16) {
-        // d_state 64 / 128: 16 lanes per channel of 4 / 8 states, 8 channels per CTA
+        // d_state 64 / 128: 16 lanes per channel of 4 / 8 states, 8 channels per CTA; with
+        // A per head (and input-dependent B, C) each lane serves two channels, which share
+        // its B/C loads (16 channels per CTA). SSM_CHANNELS_PER_LANE=1 keeps one.
         s = 16;
         np = ns / 16;
+        kc = (a->a_heads > 0 && !a->bc_shared) ? env_int("SSM_CHANNELS_PER_LANE", 2) : 1;
+        if (kc != 1 && kc != 2) kc = 2;
     } else if (ns == 16) {
         // Batch rows with enough channels for two 32-channel CTAs per SM: 4 lanes per
         // channel (4 states each) in CTAs of 4 scan warps. Fewer channels: 8 lanes per

@@ -104,3 +104,15 @@ def test_one_head_spans_all_channels():
     """a_heads = 1: every channel shares one decay."""
     inp = _inputs(1, 32, 100, 64, "f32", 1, False, seed=94)
     _check(_gpu(inp, "f32"), _ref(inp), "f32", "one head")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("per_lane", ["1", "2"])
+@pytest.mark.parametrize("mode", ["fwd", "bidir"])
+def test_heads_channels_per_lane(monkeypatch, dtype, N, per_lane, mode):
+    """d_state 64 / 128 with A per head: one or two channels per lane (the default, which
+    shares each lane's B/C loads between its channels), on a ragged channel count."""
+    monkeypatch.setenv("SSM_CHANNELS_PER_LANE", per_lane)
+    inp = _inputs(2, 40, 150, N, dtype, 4, False, bidir=mode == "bidir", seed=95)
+    _check(_gpu(inp, dtype, mode=mode), _ref(inp, mode), dtype, f"per_lane={per_lane}")
