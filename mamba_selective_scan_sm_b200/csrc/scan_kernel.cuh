@@ -72,8 +72,10 @@ struct ScanCfg {
     static constexpr int NT = SCAN_THREADS + kProThreads;   // threads per CTA
     // CTAs per SM the launch bounds ask for: three of 6 warps (96 registers per
     // thread), three of 4 warps with two channels per lane (168), five of 4 warps (96);
-    // two for d_state 64 / 128 (their B/C tiles take up to 113 KB of shared memory)
-    static constexpr int MIN_CTAS = NP * S > 16 ? 2 : (SW == 4 ? 3 : (KC == 2 ? 3 : 5));
+    // two for d_state 64 / 128 (their B/C tiles take up to 127 KB of shared memory), one
+    // of 10 warps with 8 scan warps
+    static constexpr int MIN_CTAS =
+        SW == 8 ? 1 : NP * S > 16 ? 2 : (SW == 4 ? 3 : (KC == 2 ? 3 : 5));
     static constexpr int NS = NP * S;            // padded state count
     static constexpr int ES = sizeof(T);
     static constexpr int TT = 64 / ES;           // tile length: 32 (bf16) / 16 (fp32) steps

@@ -20,7 +20,8 @@ namespace ssm {
     X(4, 16, 1, 4, 1, 1)     \
     X(8, 16, 1, 4, 1, 1)     \
     X(4, 16, 2, 4, 0, 2)     \
-    X(8, 16, 2, 4, 0, 2)
+    X(8, 16, 2, 4, 0, 2)     \
+    X(8, 16, 2, 8, 0, 2)
 
 // One scan pass with split `v`: one sequence per row in the (batch, dim, seqlen)
 // layout (scan_bf16.cu / scan_f32.cu), packed sequences / channel-last

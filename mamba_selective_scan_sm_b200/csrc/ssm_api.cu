@@ -191,6 +191,10 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         np = ns / 16;
         kc = (a->a_heads > 0 && !a->bc_shared) ? env_int("SSM_CHANNELS_PER_LANE", 2) : 1;
         if (kc != 1 && kc != 2) kc = 2;
+        // d_state 128 with two channels per lane: the staged tiles take 127 KB per CTA of
+        // 4 scan warps, so one CTA fits an SM; CTAs of 8 scan warps (32 channels) keep 10
+        // warps per SM instead of 6 (SSM_SCAN_WARPS=4 keeps the smaller CTA)
+        if (ns == 128 && kc == 2) sw = env_int("SSM_SCAN_WARPS", 8) == 4 ? 4 : 8;
     } else if (ns == 16) {
         // Batch rows with enough channels for two 32-channel CTAs per SM: 4 lanes per
         // channel (4 states each) in CTAs of 4 scan warps. Fewer channels: 8 lanes per

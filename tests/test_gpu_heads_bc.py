@@ -116,3 +116,13 @@ def test_heads_channels_per_lane(monkeypatch, dtype, N, per_lane, mode):
     monkeypatch.setenv("SSM_CHANNELS_PER_LANE", per_lane)
     inp = _inputs(2, 40, 150, N, dtype, 4, False, bidir=mode == "bidir", seed=95)
     _check(_gpu(inp, dtype, mode=mode), _ref(inp, mode), dtype, f"per_lane={per_lane}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("scan_warps", ["4", "8"])
+def test_heads_large_state_cta_sizes(monkeypatch, dtype, scan_warps):
+    """d_state 128, A per head, two channels per lane: CTAs of 4 scan warps (16 channels)
+    and of 8 (32 channels, the default), with a channel count that leaves a partial CTA."""
+    monkeypatch.setenv("SSM_SCAN_WARPS", scan_warps)
+    inp = _inputs(2, 72, 130, 128, dtype, 6, False, seed=96)
+    _check(_gpu(inp, dtype, chunks=2), _ref(inp), dtype, f"scan warps {scan_warps}")
