@@ -117,7 +117,7 @@ def fp32_ops(w) -> int:
 KERNEL_SOURCES = {
     "scan": ("scan_kernel.cuh", "device_common.cuh", "scan_params.h", "scan_launch.cuh",
              "scan_variants.h", "scan_bf16.cu", "scan_f32.cu", "scan_bf16_ext.cu",
-             "scan_f32_ext.cu", "kernels.cu", "ssm_api.cu"),
+             "scan_f32_ext.cu", "scan_bf16_m2.cu", "scan_f32_m2.cu", "kernels.cu", "ssm_api.cu"),
     "decode": ("decode_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
                "ssm_api.cu"),
     "conv": ("conv_kernel.cuh", "device_common.cuh", "scan_params.h", "kernels.cu",
