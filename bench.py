@@ -299,7 +299,9 @@ class ConvWorkload:
 
     One step's 100 MB (x read, y written) would fit the 126 MB L2, so steps rotate over
     SETS independent input/output pairs: a step's tensors were last touched SETS - 1
-    steps earlier, with ~200 MB of other traffic in between."""
+    steps earlier, with ~200 MB of other traffic in between. The launch (~21 us) is
+    shorter than the binding's host-side call, so each set's launch is captured once in
+    a CUDA graph and a step replays it (the end-to-end leg calls the binding itself)."""
 
     SETS = 3
 
@@ -319,11 +321,25 @@ class ConvWorkload:
         self.k = 0
         self.launches_per_step = 1
         self.h = None
+        self.launch(0)                                  # load the kernel outside the capture
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        self.graphs = []
+        for i in range(self.SETS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+                self.launch(i)
+            self.graphs.append(g)
+        torch.cuda.current_stream().wait_stream(side)
+
+    def launch(self, i):
+        self.ssm.ssm_causal_conv1d_fwd(self.xs[i], self.cw, self.cb, True, out=self.outs[i])
 
     def step(self):
         i = self.k % self.SETS
         self.k += 1
-        self.ssm.ssm_causal_conv1d_fwd(self.xs[i], self.cw, self.cb, True, out=self.outs[i])
+        self.graphs[i].replay()
 
     def e2e_setup(self):
         self.h = self.x.cpu().pin_memory()
@@ -333,8 +349,9 @@ class ConvWorkload:
 
     def e2e_step(self):
         i = self.k % self.SETS
+        self.k += 1
         self.xs[i].copy_(self.h, non_blocking=True)
-        self.step()
+        self.launch(i)
         self.hout.copy_(self.outs[i], non_blocking=True)
 
     def elems(self):
