@@ -239,3 +239,21 @@ def test_wait_selftest_rejects_limits_out_of_range(lib):
     assert lib.ssm_wait_selftest(10, None) == _abi.STATUS_CODE["SSM_ERR_BAD_SHAPE"]
     assert lib.ssm_wait_selftest(10 ** 10, None) == _abi.STATUS_CODE["SSM_ERR_BAD_SHAPE"]
 
+
+
+def test_binding_workspace_query_for_heads_and_time_invariant_bc(lib):
+    """The binding's host-only workspace query with A given per head (d_state must then
+    be passed) and with time-invariant B/C; CPU tensors are enough (shapes only)."""
+    import torch
+    import mamba_selective_scan_sm_b200 as ssm
+    u = torch.empty(1, 64, 4096, dtype=torch.bfloat16)
+    A_heads = torch.empty(8)
+    with pytest.raises(ValueError):
+        ssm.ssm_selective_scan_workspace_size(u, A_heads, num_chunks=4)
+    n = ssm.ssm_selective_scan_workspace_size(u, A_heads, num_chunks=4, dstate=128)
+    assert n == 3 * 64 * 128 * 8                      # (chunks-1) x rows x 128 x (P, S)
+    A = torch.empty(64, 16)
+    n = ssm.ssm_selective_scan_workspace_size(u, A, num_chunks=4, bc_shared=True)
+    assert n == 3 * 64 * 16 * 8
+    with pytest.raises(RuntimeError):                 # 64 channels are not 5 whole heads
+        ssm.ssm_selective_scan_workspace_size(u, torch.empty(5), num_chunks=4, dstate=16)
