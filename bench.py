@@ -362,8 +362,8 @@ class DecodeWorkload:
     """The decode configuration: 64 successive single-token updates of every (b, d) row.
 
     One bench step replays a CUDA graph of the 64 token launches (no host launch
-    overhead between tokens). The state of one layer (84 MB fp32 + 10.5 MB conv state)
-    would fit the 126 MB L2, so the tokens rotate over LAYERS independent state
+    overhead between tokens). The state of one layer (at B256 D5120 N16: 84 MB fp32 + 10.5
+    MB conv state) would fit the 126 MB L2, so the tokens rotate over LAYERS independent state
     buffers (one per layer of a model): a token's state was last touched LAYERS - 1
     launches earlier, and ~190 MB of other traffic has gone through L2 since."""
 
@@ -373,7 +373,8 @@ class DecodeWorkload:
         import torch
         import mamba_selective_scan_sm_b200 as ssm
         self.w, self.torch, self.ssm = w, torch, ssm
-        inp = synth.decode_inputs(w.batch, w.dim, w.dstate, w.steps, 4, w.dtype, seed=0)
+        inp = synth.decode_inputs(w.batch, w.dim, w.dstate, w.steps, 4, w.dtype, seed=0,
+                                  a_heads=w.extra.get("a_heads", 0))
         self.host_inp = inp
         bf = torch.bfloat16
         st = torch.from_numpy(inp["state"]).to(device)
@@ -429,7 +430,8 @@ def oracle_sample(w, seconds=10.0):
     """Time the CPU oracle on a bounded sample of the workload; returns (elems/s, desc, cores)."""
     import oracle
     if w.name.startswith("decode"):
-        inp = synth.decode_inputs(1, 256, w.dstate, 4, 4, w.dtype, seed=0)
+        inp = synth.decode_inputs(1, 256, w.dstate, 4, 4, w.dtype, seed=0,
+                                  a_heads=4 if w.extra.get("a_heads") else 0)
         t0 = time.perf_counter()
         n = 0
         st, cs = inp["state"], inp["conv_state"]
@@ -537,8 +539,10 @@ def config_of(w, args):
         c["l2"] = (f"steps rotate over {ConvWorkload.SETS} input/output pairs "
                    f"({ConvWorkload.SETS * ab / 1e6:.0f} MB > 126 MB L2)")
     elif w.name.startswith("decode"):
+        es = 2 if w.dtype == "bf16" else 4
+        layer_mb = w.batch * w.dim * (w.dstate * 4 + w.conv_width * es) / 1e6   # SSM + conv state
         c["l2"] = (f"state rotated over {DecodeWorkload.LAYERS} layers "
-                   f"({DecodeWorkload.LAYERS * 94.5:.0f} MB of state > 126 MB L2): no step "
+                   f"({DecodeWorkload.LAYERS * layer_mb:.0f} MB of state > 126 MB L2): no step "
                    "finds its state in L2")
     else:
         c["l2"] = ("inputs larger than L2 ({:.0f} MB/step > 126 MB)".format(ab / 1e6)

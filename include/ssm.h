@@ -67,7 +67,7 @@ extern "C" {
 #define SSM_API
 #endif
 
-#define SSM_ABI_VERSION 3
+#define SSM_ABI_VERSION 4
 #define SSM_MAX_DSTATE 16        /* decode (ssm_selective_state_update) */
 #define SSM_MAX_SCAN_DSTATE 128  /* scan (ssm_selective_scan_fwd) */
 #define SSM_MAX_CONV_WIDTH 4
@@ -233,6 +233,41 @@ SSM_API ssm_status_t ssm_selective_state_update(float* state, void* conv_state, 
                                         int32_t conv_width, void* out, int64_t batch,
                                         int64_t dim, int64_t dstate, ssm_dtype_t dtype,
                                         ssm_stream_t stream);
+
+/* Arguments of ssm_selective_state_update_ex. Zero-initialise, then fill. The fields
+ * mean what the arguments of ssm_selective_state_update mean, plus: */
+typedef struct {
+    ssm_dtype_t dtype;
+    int64_t batch, dim;
+    int64_t dstate;           /* 1..SSM_MAX_SCAN_DSTATE */
+    float* state;             /* (batch, dim, dstate) fp32, in/out */
+    void* conv_state;         /* (batch, dim, conv_width) in dtype, in/out; or NULL */
+    const void* x;            /* (batch, dim) */
+    const void* dt;           /* (batch, dim) */
+    const float* A;           /* (dim, dstate), or (a_heads) with a_heads > 0 */
+    const void* B_t;          /* (batch, dstate) */
+    const void* C_t;          /* (batch, dstate) */
+    const float* D;           /* (dim) or NULL */
+    const void* z;            /* (batch, dim) or NULL */
+    const float* dt_bias;     /* (dim) or NULL */
+    int32_t dt_softplus;
+    const float* conv_weight; /* (dim, conv_width) or NULL */
+    const float* conv_bias;   /* (dim) or NULL */
+    int32_t conv_width;
+    void* out;                /* (batch, dim) */
+    /* A as one scalar per head, heads contiguous over the channels (the same reading as
+     * ssm_scan_args_t.a_heads): every state of a channel of head h decays by
+     * exp(delta * A[h]); 0: A is (dim, dstate). */
+    int32_t a_heads;
+} ssm_update_args_t;
+
+/* The decode step of ssm_selective_state_update, for d_state up to SSM_MAX_SCAN_DSTATE
+ * and A per head (the step method of the scan's per-head form). With d_state <= 16 and
+ * a_heads = 0 it runs the same kernels as ssm_selective_state_update. Errors as there;
+ * SSM_ERR_BAD_SHAPE also for a_heads < 0 or not dividing dim; SSM_ERR_ALIAS also when
+ * conv_state overlaps state. */
+SSM_API ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* args,
+                                                   ssm_stream_t stream);
 
 /*
  * Selective-scan forward that allocates nothing (the pages have no counterpart:

@@ -238,13 +238,26 @@ def ssm_selective_state_update(state, conv_state, x, dt, A, B, C, D=None, z=None
                                dt_softplus=True, conv_weight=None, conv_bias=None, *, out=None,
                                stream=None):
     """One decode step, in place on ``state`` (batch, dim, dstate) fp32 and ``conv_state``
-    (batch, dim, width). x, dt, z (batch, dim); B, C (batch, dstate). Returns y (batch, dim)."""
+    (batch, dim, width). x, dt, z (batch, dim); B, C (batch, dstate); A (dim, dstate), or
+    (nheads,) for one scalar per head; dstate up to 128. Returns y (batch, dim)."""
     torch = _torch()
     lib = _abi.load()
     if out is None:
         out = torch.empty_like(x)
     batch, dim, dstate = state.shape
     width = conv_weight.shape[1] if conv_weight is not None else 0
+    if A.dim() == 1 or dstate > 16:
+        # A per head (a 1-D tensor, one scalar per head) or d_state above 16
+        a = _abi.UpdateArgs()
+        a.dtype, a.batch, a.dim, a.dstate = _dtype_code(x), batch, dim, dstate
+        a.state, a.conv_state, a.x, a.dt = _fp32(state, "state"), _ptr(conv_state), _ptr(x), _ptr(dt)
+        a.A, a.B_t, a.C_t, a.D = _fp32(A, "A"), _ptr(B), _ptr(C), _fp32(D, "D")
+        a.z, a.dt_bias, a.dt_softplus = _ptr(z), _fp32(dt_bias, "dt_bias"), int(bool(dt_softplus))
+        a.conv_weight, a.conv_bias = _fp32(conv_weight, "conv_weight"), _fp32(conv_bias, "conv_bias")
+        a.conv_width, a.out = width, _ptr(out)
+        a.a_heads = A.shape[0] if A.dim() == 1 else 0
+        _abi.check(lib, lib.ssm_selective_state_update_ex(ctypes.byref(a), _stream(stream)))
+        return out
     _abi.check(lib, lib.ssm_selective_state_update(
         _fp32(state, "state"), _ptr(conv_state), _ptr(x), _ptr(dt), _fp32(A, "A"), _ptr(B),
         _ptr(C), _fp32(D, "D"), _ptr(z), _fp32(dt_bias, "dt_bias"), int(bool(dt_softplus)),

@@ -19,10 +19,11 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTS = (
     "ssm_abi_version", "ssm_status_string", "ssm_last_error_detail", "ssm_causal_conv1d_fwd",
     "ssm_selective_scan_workspace_size", "ssm_selective_scan_fwd", "ssm_selective_state_update",
-    "ssm_device_error", "ssm_selective_scan_fwd_noalloc", "ssm_wait_selftest",
+    "ssm_selective_state_update_ex", "ssm_device_error", "ssm_selective_scan_fwd_noalloc",
+    "ssm_wait_selftest",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
-ABI_VERSION = 3            # SSM_ABI_VERSION of include/ssm.h this mirror follows
+ABI_VERSION = 4            # SSM_ABI_VERSION of include/ssm.h this mirror follows
 
 _P = ctypes.c_void_p
 _FP = ctypes.POINTER(ctypes.c_float)
@@ -47,6 +48,18 @@ class ScanArgs(ctypes.Structure):
         ("channel_last", _I32), ("stride_u", _I64), ("stride_delta", _I64), ("stride_z", _I64),
         ("stride_out", _I64), ("stride_B", _I64), ("stride_C", _I64),
         ("a_heads", _I32), ("bc_shared", _I32),
+    ]
+
+
+class UpdateArgs(ctypes.Structure):
+    """Mirror of ssm_update_args_t (field order and types as in include/ssm.h)."""
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("batch", _I64), ("dim", _I64), ("dstate", _I64),
+        ("state", _P), ("conv_state", _P), ("x", _P), ("dt", _P), ("A", _P), ("B_t", _P),
+        ("C_t", _P), ("D", _P), ("z", _P), ("dt_bias", _P), ("dt_softplus", _I32),
+        ("conv_weight", _P), ("conv_bias", _P), ("conv_width", _I32), ("out", _P),
+        ("a_heads", _I32),
     ]
 
 
@@ -84,6 +97,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssm_selective_state_update.restype = ctypes.c_int
     lib.ssm_selective_state_update.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _P,
                                                _P, _I32, _P, _I64, _I64, _I64, ctypes.c_int, _P]
+    lib.ssm_selective_state_update_ex.restype = ctypes.c_int
+    lib.ssm_selective_state_update_ex.argtypes = [ctypes.POINTER(UpdateArgs), _P]
     lib.ssm_selective_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _P]
     lib.ssm_device_error.restype = ctypes.c_int

@@ -468,4 +468,105 @@ __global__ void __launch_bounds__(256) decode_bulk_kernel(const DecodeParams p) 
     }
 }
 
+
+// Decode step for d_state up to 128 and for A given per head. LPR lanes serve one (b, d)
+// row, 16 states each (lane q of the row holds states 16q .. 16q + 15, four float4s), so
+// a warp holds 32 / LPR rows (4 at d_state 128, 32 at d_state <= 16) and the per-row
+// work (conv, softplus, gate, parameter loads) is shared by 16 states of every lane.
+// With A per head the row's decay exp(delta * A_h) is one exp for all its states. Every
+// lane takes part in the row's shuffle reduction, so no lane leaves early. Grid: x =
+// groups of 8 * 32 / LPR channels, y (+ 65535 * z) = batch row: no index divisions.
+template <typename T, int LPR>
+__global__ void __launch_bounds__(256) decode_warp_kernel(const DecodeParams p) {
+    using E = Elem<T>;
+    constexpr int RPW = 32 / LPR;
+    constexpr int NPL = 16;                                // states per lane
+    const int lane = threadIdx.x & 31;
+    const int dd = (blockIdx.x * 8 + (threadIdx.x >> 5)) * RPW + lane / LPR;
+    const int64_t b0 = (int64_t)blockIdx.z * 65535 + blockIdx.y;
+    const int q = lane % LPR;
+    const bool live = dd < p.dim && b0 * p.dim < p.rows;
+    const int d = live ? dd : 0;                           // dead lanes read row 0, store nothing
+    const int64_t bb = live ? b0 : 0;
+    const int64_t rr = bb * p.dim + d;
+    const int N = p.dstate;
+    const int n0 = NPL * q;
+    // the state row first: its loads are the long ones and depend on nothing else (the
+    // host rejects a conv state that overlaps the SSM state)
+    float* st = p.state + rr * N;
+    float h[NPL];
+#pragma unroll
+    for (int g = 0; g < NPL / 4; ++g) {
+        const int n = n0 + 4 * g;
+        if (p.vec && n + 3 < N) {                          // dstate % 4 == 0, aligned rows
+            const float4 v = *reinterpret_cast<const float4*>(st + n);
+            h[4 * g] = v.x; h[4 * g + 1] = v.y; h[4 * g + 2] = v.z; h[4 * g + 3] = v.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[4 * g + i] = n + i < N ? st[n + i] : 0.f;
+        }
+    }
+    const T* Bt = static_cast<const T*>(p.Bt) + bb * N;
+    const T* Ct = static_cast<const T*>(p.Ct) + bb * N;
+    const float xt = E::to_f(static_cast<const T*>(p.x)[rr]);
+    float dl = E::to_f(static_cast<const T*>(p.dt)[rr]) + (p.dt_bias ? p.dt_bias[d] : 0.f);
+    float xc = xt;
+    if (p.conv_w) {
+        // the window after the shift: conv_state[1 .. W-1], then x_t (newest last)
+        T* cs = static_cast<T*>(p.conv_state) + rr * p.conv_width;
+        float win[4];
+        float acc = p.conv_b ? p.conv_b[d] : 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k < p.conv_width) {
+                win[k] = k < p.conv_width - 1 ? E::to_f(cs[k + 1]) : xt;
+                acc = fmaf(p.conv_w[(int64_t)d * p.conv_width + k], win[k], acc);
+            }
+        }
+        xc = silu(acc);
+        __syncwarp();                                      // the row's lanes have read cs
+        if (live && q == 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < p.conv_width) cs[k] = E::from_f(win[k]);   // exact: values of T
+        }
+    }
+    if (p.softplus) dl = softplus(dl);
+    const float du = dl * xc;
+    const bool heads = p.head_dim != 0;
+    const float dAh = heads ? ex2(dl * p.A[d / p.head_dim] * kLog2e) : 0.f;
+    const float* Ar = p.A + (int64_t)d * N;
+    float y = 0.f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int n = n0 + i;
+        if (n < N) {
+            const float dA = heads ? dAh : ex2(dl * Ar[n] * kLog2e);
+            h[i] = fmaf(dA, h[i], du * E::to_f(Bt[n]));
+            y = fmaf(E::to_f(Ct[n]), h[i], y);
+        }
+    }
+    if (live) {
+#pragma unroll
+        for (int g = 0; g < NPL / 4; ++g) {
+            const int n = n0 + 4 * g;
+            if (p.vec && n + 3 < N) {
+                *reinterpret_cast<float4*>(st + n) =
+                    make_float4(h[4 * g], h[4 * g + 1], h[4 * g + 2], h[4 * g + 3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (n + i < N) st[n + i] = h[4 * g + i];
+            }
+        }
+    }
+#pragma unroll
+    for (int m = LPR / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+    if (live && q == 0) {
+        if (p.D) y = fmaf(p.D[d], xc, y);
+        if (p.z) y *= silu(E::to_f(static_cast<const T*>(p.z)[rr]));
+        static_cast<T*>(p.out)[rr] = E::from_f(y);
+    }
+}
+
 }  // namespace ssm

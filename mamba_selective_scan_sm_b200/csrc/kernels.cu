@@ -122,6 +122,28 @@ cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_
     return cudaGetLastError();
 }
 
+cudaError_t launch_decode_warp(int es, const DecodeParams& p, cudaStream_t st) {
+    // lanes per row: 16 states per lane
+    const int lpr = p.dstate <= 16 ? 1 : p.dstate <= 32 ? 2 : p.dstate <= 64 ? 4 : 8;
+    const int per_block = 8 * (32 / lpr);                       // channels per 8-warp block
+    const int64_t batch = p.rows / p.dim;
+    const int64_t bz = (batch + 65534) / 65535;
+    if (bz > 65535) return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)((p.dim + per_block - 1) / per_block),
+                    (unsigned)(batch < 65535 ? batch : 65535), (unsigned)bz);
+#define SSM_WARP_LPR(T_, L_) \
+    if (lpr == L_) { decode_warp_kernel<T_, L_><<<grid, 256, 0, st>>>(p); return cudaGetLastError(); }
+    if (es == 2) {
+        SSM_WARP_LPR(__nv_bfloat16, 1) SSM_WARP_LPR(__nv_bfloat16, 2)
+        SSM_WARP_LPR(__nv_bfloat16, 4) SSM_WARP_LPR(__nv_bfloat16, 8)
+    } else {
+        SSM_WARP_LPR(float, 1) SSM_WARP_LPR(float, 2) SSM_WARP_LPR(float, 4)
+        SSM_WARP_LPR(float, 8)
+    }
+#undef SSM_WARP_LPR
+    return cudaErrorInvalidValue;
+}
+
 // One thread waits, bounded by limit_ns, on an mbarrier that nothing arrives at: the
 // wait runs out, sets the device error word and the kernel returns (a self-test of the
 // failure path every kernel's waits share).

@@ -36,6 +36,9 @@ cudaError_t launch_conv_tail(int elem_size, const ConvTailParams& p, cudaStream_
 
 cudaError_t launch_decode(int elem_size, int dstate, const DecodeParams& p, cudaStream_t stream);
 
+// Decode step for d_state up to 128 and A per head (p.head_dim), 16 states per lane.
+cudaError_t launch_decode_warp(int elem_size, const DecodeParams& p, cudaStream_t stream);
+
 // Replace the calling thread's ssm_last_error_detail() text.
 void set_error_detail(const char* text);
 

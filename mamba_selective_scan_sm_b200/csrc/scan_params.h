@@ -92,6 +92,7 @@ struct DecodeParams {
     int vec;            // dstate == 16 and state / A rows 16-byte aligned
     int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
     int stream;         // streaming variant: dstate 16, dim % 128 == 0, 16-byte aligned bases
+    int head_dim;       // A one scalar per head (A[d / head_dim]); 0: A is (dim, dstate)
 };
 
 }  // namespace ssm

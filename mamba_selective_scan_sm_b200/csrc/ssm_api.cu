@@ -617,6 +617,80 @@ ssm_status_t ssm_selective_state_update(float* state, void* conv_state, const vo
     return ok();
 }
 
+ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* a, ssm_stream_t stream) {
+    if (!a) return fail(SSM_ERR_NULL_ARG, "args is NULL");
+    if (a->a_heads < 0 || (a->a_heads > 0 && a->dim > 0 && a->dim % a->a_heads != 0))
+        return fail(SSM_ERR_BAD_SHAPE, "a_heads %d must be 0 or divide dim %lld", a->a_heads,
+                    (long long)a->dim);
+    if (a->dstate <= SSM_MAX_DSTATE && a->a_heads == 0)
+        return ssm_selective_state_update(a->state, a->conv_state, a->x, a->dt, a->A, a->B_t,
+                                          a->C_t, a->D, a->z, a->dt_bias, a->dt_softplus,
+                                          a->conv_weight, a->conv_bias, a->conv_width, a->out,
+                                          a->batch, a->dim, a->dstate, a->dtype, stream);
+    if (a->dtype != SSM_F32 && a->dtype != SSM_BF16)
+        return fail(SSM_ERR_BAD_DTYPE, "dtype %d is not SSM_F32 or SSM_BF16", (int)a->dtype);
+    if (a->batch < 0 || a->dim < 0) return fail(SSM_ERR_BAD_SHAPE, "negative size");
+    if (a->dstate < 1 || a->dstate > SSM_MAX_SCAN_DSTATE)
+        return fail(SSM_ERR_BAD_SHAPE, "dstate %lld outside 1..%d", (long long)a->dstate,
+                    SSM_MAX_SCAN_DSTATE);
+    if (a->conv_weight && (a->conv_width < 1 || a->conv_width > SSM_MAX_CONV_WIDTH))
+        return fail(SSM_ERR_BAD_SHAPE, "conv_width %d outside 1..%d", a->conv_width,
+                    SSM_MAX_CONV_WIDTH);
+    if (a->dim > 0x3fffffffLL) return fail(SSM_ERR_BAD_SHAPE, "dim must be below 2^30");
+    const int64_t rows = a->batch * a->dim;
+    if (rows == 0) return ok();
+    if (rows > (int64_t)1 << 28)
+        return fail(SSM_ERR_BAD_SHAPE, "batch * dim = %lld exceeds 2^28", (long long)rows);
+    struct { const void* p; const char* n; } req[] = {
+        {a->state, "state"}, {a->x, "x"}, {a->dt, "dt"}, {a->A, "A"}, {a->B_t, "B_t"},
+        {a->C_t, "C_t"}, {a->out, "out"}};
+    for (auto& r : req)
+        if (!r.p) return fail(SSM_ERR_NULL_ARG, "%s is NULL", r.n);
+    if (a->conv_weight && !a->conv_state) return fail(SSM_ERR_NULL_ARG, "conv_state is NULL");
+    const int es = elem_size(a->dtype);
+    struct { const void* p; size_t al; const char* n; } al[] = {
+        {a->state, 4, "state"}, {a->conv_state, (size_t)es, "conv_state"}, {a->x, (size_t)es, "x"},
+        {a->dt, (size_t)es, "dt"}, {a->A, 4, "A"}, {a->B_t, (size_t)es, "B_t"},
+        {a->C_t, (size_t)es, "C_t"}, {a->D, 4, "D"}, {a->z, (size_t)es, "z"},
+        {a->dt_bias, 4, "dt_bias"}, {a->conv_weight, 4, "conv_weight"},
+        {a->conv_bias, 4, "conv_bias"}, {a->out, (size_t)es, "out"}};
+    for (auto& x : al)
+        if (x.p && !aligned(x.p, x.al))
+            return fail(SSM_ERR_MISALIGNED, "%s is not %zu-byte aligned", x.n, x.al);
+    const size_t on = (size_t)rows * es;
+    if (overlap(a->out, on, a->x, on) || overlap(a->out, on, a->dt, on) ||
+        overlap(a->out, on, a->z, on) ||
+        overlap(a->out, on, a->state, (size_t)rows * a->dstate * 4))
+        return fail(SSM_ERR_ALIAS, "out overlaps an input");
+    if (a->conv_weight && overlap(a->conv_state, (size_t)rows * a->conv_width * es, a->state,
+                                  (size_t)rows * a->dstate * 4))
+        return fail(SSM_ERR_ALIAS, "conv_state overlaps state");
+    ssm::DecodeParams p{};
+    p.state = a->state;
+    p.conv_state = a->conv_weight ? a->conv_state : nullptr;
+    p.x = a->x;
+    p.dt = a->dt;
+    p.A = a->A;
+    p.Bt = a->B_t;
+    p.Ct = a->C_t;
+    p.D = a->D;
+    p.z = a->z;
+    p.dt_bias = a->dt_bias;
+    p.conv_w = a->conv_weight;
+    p.conv_b = a->conv_weight ? a->conv_bias : nullptr;
+    p.out = a->out;
+    p.rows = rows;
+    p.dim = (int)a->dim;
+    p.dstate = (int)a->dstate;
+    p.conv_width = a->conv_weight ? a->conv_width : 0;
+    p.softplus = a->dt_softplus ? 1 : 0;
+    p.vec = a->dstate % 4 == 0 && aligned(a->state, 16);
+    p.head_dim = a->a_heads > 0 ? (int)(a->dim / a->a_heads) : 0;
+    cudaError_t e = ssm::launch_decode_warp(es, p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+    return ok();
+}
+
 ssm_status_t ssm_wait_selftest(uint64_t limit_ns, ssm_stream_t stream) {
     if (limit_ns < 1000 || limit_ns > 1000000000ull)
         return fail(SSM_ERR_BAD_SHAPE, "limit_ns %llu outside 1 us .. 1 s",

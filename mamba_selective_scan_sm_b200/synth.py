@@ -111,6 +111,9 @@ WORKLOADS = {
                       bidirectional=True),
     "decode": Workload("decode B256 D5120 N16 bf16 x64 steps", 256, 5120, 1, 16, "bf16",
                        conv_width=4, steps=64),
+    "decode_h128": Workload("decode B256 D1536 (24 heads x 64) N128 bf16 x64 steps: A one scalar "
+                            "per head (Mamba-2-130M shape)", 256, 1536, 1, 128, "bf16",
+                            conv_width=4, steps=64, extra={"a_heads": 24}),
     "conv": Workload("causal conv1d + SiLU B8 D1536 L2048 bf16 width 4", 8, 1536, 2048, 16,
                      "bf16", conv_width=4, extra={"conv_only": True}),
     "m130_cl": Workload("Mamba-130M layer in the block's layout B8 L2048 D1536 N16 bf16 + conv4: "
@@ -179,12 +182,13 @@ def scan_inputs(batch: int, dim: int, seqlen: int, dstate: int = 16, dtype: str 
 
 
 def decode_inputs(batch: int, dim: int, dstate: int = 16, steps: int = 1, conv_width: int = 4,
-                  dtype: str = "bf16", seed: int = 0) -> dict:
+                  dtype: str = "bf16", seed: int = 0, a_heads: int = 0) -> dict:
     """Inputs of ``steps`` successive single-token updates.
 
     Layouts: state (batch, dim, dstate) fp32; conv_state (batch, dim, conv_width), newest
     last; per-step x, dt, z (steps, batch, dim); B_t, C_t (steps, batch, dstate);
-    A (dim, dstate); D, dt_bias, conv_b (dim); conv_w (dim, conv_width).
+    A (dim, dstate), or (a_heads,) with ``a_heads``; D, dt_bias, conv_b (dim);
+    conv_w (dim, conv_width).
     """
     out = {
         "state": normal(seed, "state", (batch, dim, dstate)),
@@ -200,4 +204,6 @@ def decode_inputs(batch: int, dim: int, dstate: int = 16, steps: int = 1, conv_w
         "conv_w": normal(seed, "conv_w", (dim, conv_width), 0.5),
         "conv_b": np.zeros(dim, dtype=np.float32),
     }
+    if a_heads:
+        out["A"] = heads_A(seed, "A_heads", a_heads)
     return out

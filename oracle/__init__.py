@@ -149,11 +149,13 @@ def state_update(state, conv_state, x, dt, A, B, C, D=None, z=None, dt_bias=None
                  dt_softplus=True, conv_w=None, conv_b=None):
     """One decode step. Returns (y (B, D), new_state, new_conv_state); inputs untouched.
 
-    state (B, D, N); conv_state (B, D, W) newest last; x, dt, z (B, D); B, C (B, N).
+    state (B, D, N); conv_state (B, D, W) newest last; x, dt, z (B, D); B, C (B, N);
+    A (D, N), or one scalar per head (nheads,).
     """
     st = _d(state).copy()
     cs = _d(conv_state).copy() if conv_state is not None else None
-    x, dt, A, B, C = _d(x), _d(dt), _d(A), _d(B), _d(C)
+    x, dt, B, C = _d(x), _d(dt), _d(B), _d(C)
+    A = _d(head_A(A, st.shape[1], st.shape[2]))
     D, z, dt_bias, conv_w, conv_b = _d(D), _d(z), _d(dt_bias), _d(conv_w), _d(conv_b)
     Bsz, Dm, N = st.shape
     W = conv_w.shape[1] if conv_w is not None else 0

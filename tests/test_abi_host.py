@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 3
+    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 4
     for code, name in _abi.STATUS.items():
         assert lib.ssm_status_string(code)
     assert lib.ssm_status_string(999) == b"unknown status"
@@ -136,19 +136,21 @@ def test_scan_continuation_arguments(lib, kw, status):
     assert lib.ssm_last_error_detail()
 
 
-def test_scan_args_layout_matches_header(tmp_path):
-    """The ctypes mirror has the C struct's size and field offsets (compiled with gcc)."""
+@pytest.mark.parametrize("mirror,ctype", [(_abi.ScanArgs, "ssm_scan_args_t"),
+                                           (_abi.UpdateArgs, "ssm_update_args_t")])
+def test_args_layout_matches_header(tmp_path, mirror, ctype):
+    """The ctypes mirrors have the C structs' sizes and field offsets (compiled with gcc)."""
     inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
-    names = [f[0] for f in _abi.ScanArgs._fields_]
-    body = "\n".join(f'printf("%zu\\n", offsetof(ssm_scan_args_t, {n}));' for n in names)
+    names = [f[0] for f in mirror._fields_]
+    body = "\n".join(f'printf("%zu\\n", offsetof({ctype}, {n}));' for n in names)
     src = tmp_path / "layout.c"
     src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"ssm.h\"\n"
                    "int main(void) {\n" + body +
-                   '\nprintf("%zu\\n", sizeof(ssm_scan_args_t));\nreturn 0;\n}\n')
+                   f'\nprintf("%zu\\n", sizeof({ctype}));\nreturn 0;\n}}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)])
     got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
-    want = [getattr(_abi.ScanArgs, n).offset for n in names] + [ctypes.sizeof(_abi.ScanArgs)]
+    want = [getattr(mirror, n).offset for n in names] + [ctypes.sizeof(mirror)]
     assert got == want
 
 
@@ -257,3 +259,36 @@ def test_binding_workspace_query_for_heads_and_time_invariant_bc(lib):
     assert n == 3 * 64 * 16 * 8
     with pytest.raises(RuntimeError):                 # 64 channels are not 5 whole heads
         ssm.ssm_selective_scan_workspace_size(u, torch.empty(5), num_chunks=4, dstate=16)
+
+
+def _update_args(**kw):
+    a = _abi.UpdateArgs()
+    a.dtype, a.batch, a.dim, a.dstate = 1, 2, 64, 128
+    for i, f in enumerate(["state", "x", "dt", "A", "B_t", "C_t", "out"]):
+        setattr(a, f, FAKE + i * (1 << 24))
+    a.dt_softplus = 1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dstate=129), "SSM_ERR_BAD_SHAPE"),
+    (dict(a_heads=5), "SSM_ERR_BAD_SHAPE"),                 # does not divide dim 64
+    (dict(a_heads=-2), "SSM_ERR_BAD_SHAPE"),
+    (dict(dtype=9), "SSM_ERR_BAD_DTYPE"),
+    (dict(x=None), "SSM_ERR_NULL_ARG"),
+    (dict(state=FAKE + 2), "SSM_ERR_MISALIGNED"),
+    (dict(out=FAKE + 1 * (1 << 24) + 64), "SSM_ERR_ALIAS"),  # inside x
+    (dict(conv_weight=FAKE + (1 << 30), conv_width=4, conv_state=FAKE + 4096),
+     "SSM_ERR_ALIAS"),                                       # conv state inside the SSM state
+    (dict(conv_weight=FAKE + (1 << 30), conv_width=4), "SSM_ERR_NULL_ARG"),
+    (dict(dstate=16, a_heads=0, conv_weight=FAKE + (1 << 30), conv_width=7), "SSM_ERR_BAD_SHAPE"),
+])
+def test_state_update_ex_rejects_bad_arguments(lib, kw, status):
+    """The decode entry for d_state up to 128 and A per head validates before launching
+    (d_state <= 16 with per-state A goes through the first entry's checks)."""
+    assert lib.ssm_selective_state_update_ex(ctypes.byref(_update_args(**kw)), None) == \
+        _abi.STATUS_CODE[status]
+    assert lib.ssm_last_error_detail()
+    assert lib.ssm_selective_state_update_ex(None, None) == _abi.STATUS_CODE["SSM_ERR_NULL_ARG"]

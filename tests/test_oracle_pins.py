@@ -254,11 +254,16 @@ def test_reverse_is_flip_forward_flip(conv):
     np.testing.assert_allclose(hr, hf, rtol=1e-14, atol=1e-14)
 
 
-def test_decode_repeated_equals_scan():
-    """L decode steps from zero state and zero conv history reproduce the fused-conv scan."""
+@pytest.mark.parametrize("N,heads", [(4, 0), (64, 3)])
+def test_decode_repeated_equals_scan(N, heads):
+    """L decode steps from zero state and zero conv history reproduce the fused-conv scan
+    (with A per head and d_state 64 too: the scan's per-head form is pinned by the dual
+    form above)."""
     rng = np.random.default_rng(7)
-    Bsz, D, L, N, W = 2, 3, 17, 4, 4
+    Bsz, D, L, W = 2, 3, 17, 4
     c = _rand_case(rng, Bsz, D, L, N, conv=W)
+    if heads:
+        c["A"] = -rng.uniform(0.2, 2.0, heads)         # one head per channel here
     y, h = oracle.selective_scan(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
                                  c["delta_bias"], True, False, c["conv_w"], c["conv_b"],
                                  return_final_state=True)
