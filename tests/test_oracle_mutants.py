@@ -139,3 +139,28 @@ def test_head_mapping_slip_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "head_A", wrong)
     with pytest.raises(AssertionError):
         pins.test_scalar_A_per_head_equals_ssd_dual_form(4, False)
+
+
+def _swapped_bidir(swap):
+    """selective_scan_bidir with the named parameters exchanged between the directions."""
+    real = oracle.selective_scan_bidir
+
+    def wrong(u, delta, A, B, C, D, z, delta_bias, A_rev, D_rev, delta_bias_rev, *a, **kw):
+        if "A" in swap:
+            A, A_rev = A_rev, A
+        if "D" in swap:
+            D, D_rev = D_rev, D
+        if "bias" in swap:
+            delta_bias, delta_bias_rev = delta_bias_rev, delta_bias
+        return real(u, delta, A, B, C, D, z, delta_bias, A_rev, D_rev, delta_bias_rev, *a, **kw)
+    return wrong
+
+
+@pytest.mark.parametrize("swap", [("A", "D", "bias"), ("A",), ("bias",), ("A", "D"), ("D", "bias")],
+                         ids=["all", "A", "bias", "A_and_D", "D_and_bias"])
+def test_bidirectional_direction_swap_is_caught(swap, monkeypatch):
+    """Routing a direction's A or dt bias to the other direction fails a pin. (D
+    alone has no wrong routing: the two skip terms add up to (D + D_rev) * u under the
+    shared gate, so exchanging only D leaves the sum unchanged.)"""
+    monkeypatch.setattr(oracle, "selective_scan_bidir", _swapped_bidir(swap))
+    assert _failing_pins(oracle._load()), f"no pin caught the exchanged {swap}"

@@ -70,6 +70,20 @@ def test_golden_scan(name):
         np.testing.assert_allclose(h, _arr(g["final_state_reverse"]), rtol=tol, atol=tol)
 
 
+def test_golden_bidirectional():
+    """Forward and reverse directions with their own A, D and dt bias, summed
+    (hand-derived fixture in which exchanging any of them changes the sum)."""
+    g = _golden("bidirectional_sum.json")
+    tol = g["tolerance"]
+    y, hf, hr = oracle.selective_scan_bidir(
+        _arr(g["u"]), _arr(g["delta"]), _arr(g["A"]), _arr(g["B"]), _arr(g["C"]), _arr(g["D"]),
+        _arr(g["z"]), _arr(g["delta_bias"]), _arr(g["A_rev"]), _arr(g["D_rev"]),
+        _arr(g["delta_bias_rev"]), g["delta_softplus"], return_final_state=True)
+    np.testing.assert_allclose(y, _arr(g["y"]), rtol=tol, atol=tol)
+    np.testing.assert_allclose(hf, _arr(g["final_state"]), rtol=tol, atol=tol)
+    np.testing.assert_allclose(hr, _arr(g["final_state_rev"]), rtol=tol, atol=tol)
+
+
 def test_golden_conv():
     g = _golden("conv_orientation.json")
     out = oracle.causal_conv1d(_arr(g["x"]), _arr(g["w"]), _arr(g["bias"]), g["apply_silu"])
