@@ -275,7 +275,10 @@ SSM_API ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* args
  * ssm_selective_scan_fwd, except that `workspace` / `workspace_bytes` are ignored:
  * the scratch the call needs (two-pass chunk summaries, the bf16 bidirectional
  * partial) lives in a fixed device array of SSM_NOALLOC_SCRATCH_BYTES compiled
- * into the library, which every GPU that loads the library holds until exit.
+ * into the library. A device holds it until exit from the moment the library's
+ * module is loaded there: with CUDA's default lazy module loading that is no later
+ * than the first no-allocation call on the device (its address lookup loads the
+ * module), with CUDA_MODULE_LOADING=EAGER when the context is created.
  * For callers that cannot call cudaMalloc (a runtime that hands out only fixed
  * buffers, a C caller with no allocator, a loop that must not risk an allocation's
  * implicit synchronisation).

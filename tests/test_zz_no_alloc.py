@@ -3,9 +3,10 @@
 The no-allocation entry point serves callers that cannot call cudaMalloc (they
 can only pass buffers they already own): its scratch is a fixed array inside the
 library. Here it must give the same results as the regular entry point given a
-caller-allocated workspace, on two calls in a row (the second call finds the
-first call's leftovers in the shared scratch), and it must refuse a call whose
-scratch would not fit, without launching anything.
+caller-allocated workspace, on two calls in a row, and it must refuse a call whose
+scratch would not fit, without launching anything. Before the compared calls, one
+call on the same shape with other inputs fills the shared scratch with unrelated
+values, so a kernel that read scratch it had not written would show it.
 
 The file is named so that pytest collects it last.
 """
@@ -76,6 +77,16 @@ def test_noalloc_matches_regular_entry_point(case):
     ws = torch.empty(max(n.value, 1), dtype=torch.uint8, device="cuda")
     a.workspace, a.workspace_bytes = ws.data_ptr(), n.value
     assert lib.ssm_selective_scan_fwd(ctypes.byref(a), _stream()) == 0
+
+    # unrelated contents in the shared scratch: the same shape with other inputs
+    other = synth.scan_inputs(B, D, L, N, dtype, conv_width=4 if case["conv"] else 0,
+                              bidirectional=case["bidir"], seed=77)
+    other["A"] = other["A"] * 0.37
+    other["delta"] = other["delta"] + 1.5
+    out_o, fs_o, fsr_o = mk()
+    c, keep3 = _args(other, dtype, conv=case["conv"], bidir=case["bidir"], chunks=case["chunks"],
+                     out=out_o, fs=fs_o, fsr=fsr_o)
+    assert lib.ssm_selective_scan_fwd_noalloc(ctypes.byref(c), _stream()) == 0
 
     # the no-allocation entry point, twice in a row on fresh outputs
     for call in range(2):
