@@ -48,6 +48,27 @@ def err_metric(g, o, dtype):
     return float(np.max(excess) / (rms if rms > 0 else 1.0))
 
 
+def plain_err(g, o):
+    """max_i |g_i - o_i| / rms(o): the error as it is, rounding of the output included."""
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    if not o.size:
+        return 0.0
+    rms = float(np.sqrt(np.mean(o * o)))
+    return float(np.max(np.abs(g - o)) / (rms if rms > 0 else 1.0))
+
+
+def max_bf16_ulp(g, o):
+    """Largest distance of a bf16 output from the rounded oracle value, in bf16 ulps."""
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    if not o.size:
+        return 0.0
+    ob = _bf16_round(o.astype(np.float32))
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ob), 2.0 ** -126))) - 7)
+    return float(np.max(np.abs(g - ob) / ulp))
+
+
 def _bf16_round(x):
     from mamba_selective_scan_sm_b200.synth import round_bf16
     return round_bf16(np.asarray(x, dtype=np.float32)).astype(np.float64)
@@ -68,10 +89,16 @@ def assert_bf16_ulp(g, o, what=""):
 
 
 def assert_close(g, o, dtype, what=""):
+    """The tolerance check; reports (pytest -s) the plain max |g - o| / rms(o) beside the
+    metric the tolerance bounds (for bf16: the error beyond the output's own rounding)."""
     e = err_metric(g, o, dtype)
     tol = F32_TOL if dtype == "f32" else BF16_TOL
+    plain = plain_err(g, o)
+    print(f"{what}: max|g-o|/rms {plain:.3e}, "
+          + (f"max rel {e:.3e}" if dtype == "f32" else
+             f"beyond bf16 rounding {e:.3e}, worst {max_bf16_ulp(g, o):.2f} bf16 ulp"))
     assert np.all(np.isfinite(np.asarray(g, dtype=np.float64))), f"{what}: non-finite output"
-    assert e <= tol, f"{what}: error {e:.3e} > {tol:.0e}"
+    assert e <= tol, f"{what}: error {e:.3e} > {tol:.0e} (max|g-o|/rms {plain:.3e})"
     return e
 
 

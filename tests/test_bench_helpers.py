@@ -52,3 +52,39 @@ def test_every_workload_has_a_config(key):
     assert bench.algorithmic_bytes(W[key]) > 0
     if W[key].extra.get("channel_last"):
         assert "layout" in c
+
+
+def test_passes_per_step_reach_the_minimum_step_time():
+    assert bench.passes_for(4.07) == 7                # 7 x 4.07 ms >= 25 ms
+    assert bench.passes_for(0.25) == 100
+    assert bench.passes_for(30.0) == 1
+    assert bench.passes_for(25.0) == 1
+    assert bench.passes_for(0.0) == 1
+    for ms in (0.03, 0.2517, 2.24, 3.3, 24.9):
+        p = bench.passes_for(ms)
+        assert p * ms >= bench.STEP_MIN_MS and (p - 1) * ms < bench.STEP_MIN_MS
+
+
+def test_recorded_traffic_reads_the_json_record(tmp_path):
+    digest = bench.kernel_source_digest("scan")
+    rec = {"rows": [{"workload": "long", "bytes": 123.0, "sources_sha256": digest},
+                    {"workload": "m130", "bytes": 7.0, "sources_sha256": "0" * 64}]}
+    p = tmp_path / "traffic.json"
+    p.write_text(__import__("json").dumps(rec))
+    assert bench.recorded_traffic("long", str(p)) == 123.0
+    assert bench.recorded_traffic("m130", str(p)) is None      # taken of other sources
+    assert bench.recorded_traffic("bidir", str(p)) is None
+    assert bench.recorded_traffic("long", str(tmp_path / "missing.json")) is None
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    import sys
+    old = sys.argv
+    sys.argv = ["bench.py"]
+    try:
+        assert bench.parse().workload == "long"
+    finally:
+        sys.argv = old
+    w = W["long"]
+    assert (w.batch, w.dim, w.seqlen, w.dstate, w.dtype, w.final_state) == (1, 5120, 65536, 16,
+                                                                           "bf16", True)
