@@ -16,7 +16,7 @@ struct ScanVariant {
     int sw;             // scan warps per CTA
     int channels;       // channels per CTA
     int threads;        // threads per CTA
-    int tile;           // time steps per tile (128 bytes of elements)
+    int tile;           // time steps per tile (64 bytes of elements)
     int halo;           // conv history elements fetched with a tile
     int smem_bytes;     // dynamic shared memory per CTA
     int min_ctas;       // CTAs per SM the launch bounds are sized for

@@ -75,7 +75,7 @@ struct ScanCfg {
     // two for d_state 64 / 128 (their B/C tiles take up to 127 KB of shared memory), one
     // of 10 warps with 8 scan warps
     static constexpr int MIN_CTAS =
-        SW == 8 ? 1 : NP * S > 16 ? 2 : (SW == 4 ? 3 : (KC == 2 ? 3 : 5));
+        SW == 8 ? 1 : NP * S > 16 ? 2 : (SW >= 3 || S == 2 || KC == 2 ? 3 : 5);
     static constexpr int NS = NP * S;            // padded state count
     static constexpr int ES = sizeof(T);
     static constexpr int TT = 64 / ES;           // tile length: 32 (bf16) / 16 (fp32) steps
@@ -90,8 +90,10 @@ struct ScanCfg {
     static constexpr int RAW_C = align_up(NS * ROWB, 1024);           // [NS][TT], swizzled
     static constexpr int RAW_X = align_up(RAW_C + NS * ROWB, 128);    // [G][TT(+HALO)]
     static constexpr int X_PITCH_MAX = (TT + HALO) * ES;
-    static constexpr int RAW_DT = align_up(RAW_X + G * X_PITCH_MAX, 128);
-    static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, 128);
+    // delta / z tiles: swizzled like B / C in the (batch, dim, seqlen) layout
+    static constexpr bool SWZDT = SSM_SWZ_DTZ != 0;
+    static constexpr int RAW_DT = align_up(RAW_X + G * X_PITCH_MAX, SWZDT ? 1024 : 128);
+    static constexpr int RAW_Z = align_up(RAW_DT + G * ROWB, SWZDT ? 1024 : 128);
     static constexpr int STAGE = align_up(RAW_Z + G * ROWB, 1024);
     // Staging buffer (fp32). P: per group of KC channels and step, KC x {delta,
     // delta*u} (one vector load per lane and step). E: per channel and step {D*u,
@@ -277,8 +279,30 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     const int d0 = blockIdx.x * G;
     const int L = p.seqlen;
     const int chunk = blockIdx.z;
-    const int cs = chunk * p.chunk_len;                    // first scan position
-    const int ce = min(cs + p.chunk_len, L);               // one past the last
+    // Scan range [cs + vbeg, ce) of this chunk, tiles from cs. Packed sequences in
+    // sequence-aligned chunks (p.seq_aligned): the chunk runs from the first sequence
+    // start at or after chunk * chunk_len to the first one at or after the next chunk's
+    // position, so it starts from a zero state and needs no carry; cs is that start
+    // rounded down to a tile, and the vbeg positions before it belong to the previous
+    // chunk (scanned by it, skipped here).
+    int cs = chunk * p.chunk_len;                          // first tile position
+    int ce = min(cs + p.chunk_len, L);                     // one past the last position
+    int vbeg = 0;
+    if (VL && p.seq_aligned) {
+        auto start_at_or_after = [&](int pos) {            // clamped to [0, L]
+            int a = 0, z = p.nseq;
+            while (a < z) {
+                const int m = (a + z) >> 1;
+                if (p.cu[m] < pos) a = m + 1; else z = m;
+            }
+            return min(max(p.cu[a], 0), L);
+        };
+        const int s0 = chunk == 0 ? 0 : start_at_or_after(cs);
+        const int s1 = chunk == p.nchunks - 1 ? L : max(start_at_or_after(ce), s0);
+        cs = s0 / TT * TT;
+        vbeg = s0 - cs;
+        ce = s1 > s0 ? s1 : cs;                             // empty: no tiles
+    }
     const int ntl = (ce - cs + TT - 1) / TT;               // tiles per direction
     const int ndir = p.mode == 2 ? 2 : 1;
     const int nt = ntl * ndir;
@@ -426,10 +450,12 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
-                reinterpret_cast<T*>(st + Cfg::RAW_DT)[r * TT + col] =
+                const int off = Cfg::SWZDT ? swz<ROWB, SWZ>(r, col * (int)sizeof(T))
+                                           : (r * TT + col) * (int)sizeof(T);
+                *reinterpret_cast<T*>(st + Cfg::RAW_DT + off) =
                     ok ? static_cast<const T*>(p.delta)[gi] : T(0.f);
                 if (has_z)
-                    reinterpret_cast<T*>(st + Cfg::RAW_Z)[r * TT + col] =
+                    *reinterpret_cast<T*>(st + Cfg::RAW_Z + off) =
                         ok ? static_cast<const T*>(p.z)[gi] : T(0.f);
             }
         };
@@ -529,18 +555,20 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 // before the tile (the conv history), reverse rows end HALO steps after it.
                 const uint4* xs = reinterpret_cast<const uint4*>(
                     st + Cfg::RAW_X + r * (CONV ? Cfg::X_PITCH_MAX : ROWB) + s0 * (int)sizeof(T));
-                const uint4* ds =
-                    reinterpret_cast<const uint4*>(st + Cfg::RAW_DT + r * ROWB + s0 * (int)sizeof(T));
-                const uint4* zs =
-                    reinterpret_cast<const uint4*>(st + Cfg::RAW_Z + r * ROWB + s0 * (int)sizeof(T));
+                // 16-byte chunk c2 of the window in the delta / z rows (swizzled or not)
+                auto dz_off = [&](int c2) {
+                    const int byte = s0 * (int)sizeof(T) + c2 * 16;
+                    return Cfg::SWZDT ? swz<ROWB, SWZ>(r, byte) : r * ROWB + byte;
+                };
                 [[maybe_unused]] uint4 xw[NXC], dw[NC], zw[NC];
                 if constexpr (!CL) {
 #pragma unroll
                     for (int c2 = 0; c2 < NXC; ++c2) xw[c2] = xs[c2];
 #pragma unroll
                     for (int c2 = 0; c2 < NC; ++c2) {
-                        dw[c2] = ds[c2];
-                        zw[c2] = has_z ? zs[c2] : make_uint4(0, 0, 0, 0);
+                        dw[c2] = *reinterpret_cast<const uint4*>(st + Cfg::RAW_DT + dz_off(c2));
+                        zw[c2] = has_z ? *reinterpret_cast<const uint4*>(st + Cfg::RAW_Z + dz_off(c2))
+                                       : make_uint4(0, 0, 0, 0);
                     }
                 }
                 // element a of the window (raw row s0 + a of the channel): from the
@@ -710,7 +738,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             ls[k].reset();
-            if (!SUMMARY && (chunk > 0 || p.h0) && chan_d(k) < p.dim) {
+            if (!SUMMARY && ((chunk > 0 && !p.seq_aligned) || p.h0) && chan_d(k) < p.dim) {
                 float hv[NP];
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
@@ -752,7 +780,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     // gate, skip term, bidirectional partial and the store of R owned outputs of the
     // lane's channel k
     auto epilogue = [&](const uint8_t* buf, int k, const float* acc, bool rv, int dir, int l0,
-                        int pos0, int nown) {
+                        int pos0, int nown, int nskip) {
         const float2* Erow =
             reinterpret_cast<const float2*>(buf + Cfg::BUF_E + (lg * KC + k) * Cfg::E_PITCH);
         float yv[R];
@@ -763,13 +791,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const float2 e = Erow[tt];
             yv[m] = (acc[m] + e.x) * e.y;
         }
-        if (chan_d(k) >= p.dim || nown <= 0) return;
+        if (chan_d(k) >= p.dim || nown <= nskip) return;
         const int tmin = rv ? l0 + TT - 1 - (pos0 + R - 1) : l0 + pos0;
         float ya[R];                                      // time-ascending order
 #pragma unroll
         for (int m = 0; m < R; ++m) ya[m] = rv ? yv[R - 1 - m] : yv[m];
         // valid ascending index range: forward [0, nown); reverse [R - nown, R)
-        const int mlo = rv ? R - nown : 0;
+        const int mlo = rv ? R - nown : nskip;   // (nskip: forward packed sequences only)
         const int mhi = rv ? R : nown;
         const int64_t gbase = chan_row(k) * L + tmin;
         // channel-last: position t of channel d at (b*L + t) * stride + d
@@ -840,6 +868,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         const int dir = tile_dir(f);
         const int i0 = cs + (f % ntl) * TT;
         const int nvalid = FULL ? TT : min(TT, ce - i0);
+        const int vlo = (!FULL && f % ntl == 0) ? vbeg : 0;   // leading steps of another chunk
         const int l0 = RV ? L - i0 - TT : i0;
         const uint8_t* Prow = buf + Cfg::BUF_P + lg * Cfg::P_PITCH;
         // packed sequences: bit tt <-> step tt starts / ends a sequence
@@ -956,7 +985,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     const int tt = RV ? TT - 1 - ii : ii;
 #pragma unroll
                     for (int k = 0; k < KC; ++k) acc[k][q] = 0.f;
-                    if (ii < nvalid) {
+                    if (ii < nvalid && ii >= vlo) {
                         float2 pd[KC];
                         float bv[NP], cv[NP];
                         load_p(tt, pd);
@@ -978,7 +1007,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             for (int k = 0; k < KC; ++k) {
                 reduce_block(acc[k]);
                 epilogue(buf, k, acc[k], RV, dir, l0, pos0,
-                         FULL ? R : max(0, min(R, nvalid - pos0)));
+                         FULL ? R : max(0, min(R, nvalid - pos0)), FULL ? 0 : max(0, vlo - pos0));
             }
         }
     };
@@ -1022,7 +1051,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         if (lane != 0) mbar_try_wait(&full_buf[f & 1], par_f);
         const uint8_t* buf = buf_of(f);
         const bool rv = tile_rev(f);
-        const bool full = cs + (f % ntl) * TT + TT <= ce;
+        const bool full = cs + (f % ntl) * TT + TT <= ce && !(f % ntl == 0 && vbeg > 0);
         if (full) {
             if (rv) scan_tile(TrueT{}, TrueT{}, f, buf);
             else scan_tile(FalseT{}, TrueT{}, f, buf);

@@ -4,15 +4,22 @@
 #include <cuda.h>
 #include <stdint.h>
 
+// The (batch, dim, seqlen) layout's delta and z tiles (64-byte rows) land with the TMA
+// 64-byte swizzle, so that the producers' 16-byte reads of consecutive rows hit distinct
+// banks (unswizzled, every other row starts on the same bank: 4-way conflicts).
+#ifndef SSM_SWZ_DTZ
+#define SSM_SWZ_DTZ 1
+#endif
+
 namespace ssm {
 
 // TMA descriptors of the streamed tensors (unused by the plain-load variant).
 struct ScanMaps {
     CUtensorMap x;    // u or pre-conv x: dims (L, D, batch), box (TT [+halo], G, 1)
-    CUtensorMap dt;   // delta:           dims (L, D, batch), box (TT, G, 1)
-    CUtensorMap z;    // gate input:      dims (L, D, batch), box (TT, G, 1)
-    CUtensorMap B;    // dims (L, N, batch), box (TT, NS, 1), 128-byte swizzle
-    CUtensorMap C;    // dims (L, N, batch), box (TT, NS, 1), 128-byte swizzle
+    CUtensorMap dt;   // delta:           dims (L, D, batch), box (TT, G, 1), 64-byte swizzle
+    CUtensorMap z;    // gate input:      dims (L, D, batch), box (TT, G, 1), 64-byte swizzle
+    CUtensorMap B;    // dims (L, N, batch), box (TT, NS, 1), swizzle spanning one tile row
+    CUtensorMap C;    // dims (L, N, batch), box (TT, NS, 1), swizzle spanning one tile row
 };
 
 struct ScanParams {
@@ -35,6 +42,7 @@ struct ScanParams {
     float* final_state[2];
     int chunk_len;          // scan positions per chunk (multiple of the tile length)
     int nchunks;
+    int seq_aligned;        // packed sequences: chunks begin at sequence starts (no carry)
     float2* summary;        // two-pass: [nchunks-1][batch*dim][NS] {prod dA, h_end}
     const float* h0;        // (batch, dim, dstate) state before position 0, or nullptr
     const void* conv_hist;  // (batch, dim, conv_width-1) inputs before position 0, or nullptr
@@ -93,6 +101,7 @@ struct DecodeParams {
     int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
     int stream;         // streaming variant: dstate 16, dim % 128 == 0, 16-byte aligned bases
     int head_dim;       // A one scalar per head (A[d / head_dim]); 0: A is (dim, dstate)
+    int vec_bc;         // B_t, C_t rows in 16-byte chunks: dstate % 16 == 0, 16-byte bases
 };
 
 }  // namespace ssm

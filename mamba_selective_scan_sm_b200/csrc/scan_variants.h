@@ -6,6 +6,8 @@
 namespace ssm {
 
 // (states per lane, lanes per channel, channels per lane, scan warps per CTA, EXT, M2):
+// 2 lanes of 8 states (the default for wide batches), 4 lanes of 4, 8 lanes of 2 in
+// CTAs of 8 or 12 channels (narrow batches);
 // EXT splits also have packed-sequence and channel-last kernels; M2 = 1 splits also have
 // kernels for A as one scalar per head and for time-invariant B/C, M2 = 2 splits for A
 // per head only. 16 lanes of 4 or 8 states cover d_state 64 and 128; with A per head
@@ -14,6 +16,8 @@ namespace ssm {
     X(4, 4, 1, 4, 1, 1)      \
     X(4, 4, 2, 2, 0, 0)      \
     X(2, 8, 1, 2, 1, 1)      \
+    X(2, 8, 1, 3, 1, 1)      \
+    X(8, 2, 1, 2, 1, 0)      \
     X(2, 8, 2, 4, 0, 0)      \
     X(2, 4, 1, 4, 1, 1)      \
     X(1, 4, 1, 4, 1, 1)      \

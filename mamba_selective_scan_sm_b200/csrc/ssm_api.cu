@@ -196,20 +196,35 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         // warps per SM instead of 6 (SSM_SCAN_WARPS=4 keeps the smaller CTA)
         if (ns == 128 && kc == 2) sw = env_int("SSM_SCAN_WARPS", 8) == 4 ? 4 : 8;
     } else if (ns == 16) {
-        // Batch rows with enough channels for two 32-channel CTAs per SM: 4 lanes per
-        // channel (4 states each) in CTAs of 4 scan warps. Fewer channels: 8 lanes per
-        // channel in CTAs of 2 scan warps (8 channels each), for more CTAs and warps.
-        // SSM_LANES_PER_CHANNEL (4, 8) and SSM_CHANNELS_PER_LANE (1, 2) pick another
-        // compiled split.
+        // Batch rows with enough channels for two 32-channel CTAs per SM: bf16, 2 lanes
+        // per channel (8 states each) in CTAs of 2 scan warps; fp32 (16-step tiles), 4
+        // lanes per channel (4 states each) in CTAs of 4 scan warps (32 channels both).
+        // Fewer channels: 8 lanes per channel (2 states each) in CTAs of 8 or 12
+        // channels, for more CTAs and warps. SSM_LANES_PER_CHANNEL (2, 4, 8) and
+        // SSM_CHANNELS_PER_LANE (1, 2) pick another compiled split.
         const bool wide = a->batch * a->dim >= 2 * 148 * 32;
-        s = env_int("SSM_LANES_PER_CHANNEL", wide ? 4 : 8);
-        if (s != 4 && s != 8) s = 4;
+        const int s_wide = a->dtype == SSM_BF16 ? 2 : 4;
+        s = env_int("SSM_LANES_PER_CHANNEL", wide ? s_wide : 8);
+        if (s != 2 && s != 4 && s != 8) s = wide ? s_wide : 8;
+        // A per head and time-invariant B/C have kernels in the 4-lane split only
+        if (s == 2 && (a->a_heads > 0 || a->bc_shared)) s = 4;
         kc = env_int("SSM_CHANNELS_PER_LANE", 1);
         if (kc != 1 && kc != 2) kc = 1;
-        if (a->seq_starts || a->channel_last || a->a_heads > 0 || a->bc_shared)
+        if (s == 2 || a->seq_starts || a->channel_last || a->a_heads > 0 || a->bc_shared)
             kc = 1;                                     // the splits compiled for those
         np = 16 / s;
-        sw = (s == 4) == (kc == 1) ? 4 : 2;
+        sw = s == 2 ? 2 : (s == 4) == (kc == 1) ? 4 : 2;
+        if (s == 8 && kc == 1) {
+            // 8 or 12 channels per CTA (2 or 3 scan warps), whichever leaves the busiest SM
+            // the fewest channels when every CTA is resident (long: 640 CTAs of 8 put 40
+            // channels on some SMs, 427 of 12 at most 36, against an average of 34.6)
+            auto busiest = [&](int64_t g) {
+                const int64_t ctas = a->batch * ((a->dim + g - 1) / g);
+                return (ctas + kNumSMs - 1) / kNumSMs * g;
+            };
+            const int64_t env_sw = env_int("SSM_SCAN_WARPS", 0);
+            sw = env_sw == 2 || env_sw == 3 ? (int)env_sw : busiest(12) < busiest(8) ? 3 : 2;
+        }
     } else if (ns == 8) {
         np = 2;
     } else {
@@ -235,8 +250,14 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
         const bool inplace = a->initial_state && a->final_state &&
                              overlap(a->final_state, stb, a->initial_state, stb);
         nch = 1;
-        if (!bidir && !inplace && ctas > 0 && 2 * ctas <= slots)
+        if (a->seq_starts) {
+            // packed sequences: chunks begin at sequence starts and need no carry, so
+            // they cost nothing extra; chunks of about 64 tiles fill the SMs and let the
+            // CTA scheduler even out the chunks' unequal lengths
+            if (ctas > 0) nch = (int)std::max<int64_t>(1, std::min<int64_t>(ntiles / 64, 4096));
+        } else if (!bidir && !inplace && ctas > 0 && 2 * ctas <= slots) {
             nch = (int)std::min<int64_t>(slots / ctas, 16);
+        }
     }
     if (nch > ntiles) nch = (int)(ntiles > 0 ? ntiles : 1);
     if (nch > 65535) nch = 65535;
@@ -245,8 +266,10 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* pl) {
     pl->nchunks = ntiles > 0 ? (int)((ntiles + tiles_per_chunk - 1) / tiles_per_chunk) : 1;
 
     const int64_t rows = a->batch * a->dim;
-    pl->summary_bytes =
-        pl->nchunks > 1 ? (size_t)(pl->nchunks - 1) * rows * ns * sizeof(float) * 2 : 0;
+    // packed sequences: sequence-aligned chunks carry nothing (no summary pass)
+    pl->summary_bytes = pl->nchunks > 1 && !a->seq_starts
+                            ? (size_t)(pl->nchunks - 1) * rows * ns * sizeof(float) * 2
+                            : 0;
     pl->partial_bytes = (bidir && a->dtype != SSM_F32) ? (size_t)rows * a->seqlen * 4 : 0;
     // layout: [summaries][pad to 256][bidirectional fp32 partial]
     pl->workspace = pl->partial_bytes ? ((pl->summary_bytes + 255) / 256) * 256 + pl->partial_bytes
@@ -431,6 +454,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
     p.final_state[1] = a->final_state_rev;
     p.chunk_len = pl.chunk_len;
     p.nchunks = pl.nchunks;
+    p.seq_aligned = packed && pl.nchunks > 1 ? 1 : 0;
     uint8_t* ws = static_cast<uint8_t*>(a->workspace);
     p.summary = pl.summary_bytes ? reinterpret_cast<float2*>(ws) : nullptr;
     p.h0 = a->initial_state;
@@ -489,9 +513,11 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
                   (sb || (map(&maps.B, a->B, N, sB, ns_pad, v.tile) &&
                           map(&maps.C, a->C, N, sC, ns_pad, v.tile)));
         } else {
+            // delta and z rows land swizzled (the kernel reads them so)
+            const CUtensorMapSwizzle dz = SSM_SWZ_DTZ ? bc : none;
             tma = encode_3d(&maps.x, es, a->u, L, D, Bn, xbox, v.channels, none) &&
-                  encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, none) &&
-                  (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, none)) &&
+                  encode_3d(&maps.dt, es, a->delta, L, D, Bn, v.tile, v.channels, dz) &&
+                  (!a->z || encode_3d(&maps.z, es, a->z, L, D, Bn, v.tile, v.channels, dz)) &&
                   (sb || (encode_3d(&maps.B, es, a->B, L, N, Bn, v.tile, v.np * v.s, bc) &&
                           encode_3d(&maps.C, es, a->C, L, N, Bn, v.tile, v.np * v.s, bc)));
         }
@@ -499,7 +525,7 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_scan_args_t* a, ssm_stream_t strea
 
     const unsigned gx = (unsigned)((a->dim + pl.v.channels - 1) / pl.v.channels);
     cudaError_t e;
-    if (pl.nchunks > 1) {
+    if (pl.nchunks > 1 && !p.seq_aligned) {
         e = ssm::launch_scan(pl.v, tma, true, packed, cl, feat, maps, p,
                              dim3(gx, (unsigned)a->batch, pl.nchunks - 1), s);
         if (e != cudaSuccess) return cuda_fail(e, "summary pass launch");
@@ -686,6 +712,7 @@ ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* a, ssm_strea
     p.softplus = a->dt_softplus ? 1 : 0;
     p.vec = a->dstate % 4 == 0 && aligned(a->state, 16);
     p.head_dim = a->a_heads > 0 ? (int)(a->dim / a->a_heads) : 0;
+    p.vec_bc = a->dstate % 16 == 0 && aligned(a->B_t, 16) && aligned(a->C_t, 16);
     cudaError_t e = ssm::launch_decode_warp(es, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return ok();

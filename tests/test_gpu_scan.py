@@ -122,11 +122,11 @@ def test_two_pass_chunk_carry(monkeypatch, dtype, reverse, chunks, per_lane):
     state_close(host(h), host(h1), "two-pass vs single-pass state")
 
 
-@pytest.mark.parametrize("lanes", ["4", "8"])
+@pytest.mark.parametrize("lanes", ["2", "4", "8"])
 @pytest.mark.parametrize("per_lane", ["1", "2"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_lane_split_variants(monkeypatch, lanes, per_lane, dtype):
-    """Every work split (4 or 8 lanes per channel, 1 or 2 channels per lane) matches."""
+    """Every work split (2, 4 or 8 lanes per channel, 1 or 2 channels per lane) matches."""
     monkeypatch.setenv("SSM_LANES_PER_CHANNEL", lanes)
     monkeypatch.setenv("SSM_CHANNELS_PER_LANE", per_lane)
     inp = synth.scan_inputs(2, 40, 300, 16, dtype, conv_width=4, seed=15)
@@ -135,6 +135,30 @@ def test_lane_split_variants(monkeypatch, lanes, per_lane, dtype):
         yo, ho = _oracle(inp, reverse=reverse, conv=True)
         assert_close_out(host(y), yo, dtype, f"y lanes={lanes}")
         state_close(host(h), ho, "final state")
+
+
+@pytest.mark.parametrize("warps", ["2", "3"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_eight_and_twelve_channel_ctas(monkeypatch, warps, dtype):
+    """8 lanes per channel in CTAs of 8 or 12 channels; dim 40 leaves the last CTA
+    partly empty (4 of 12 channels), and the chunk carry and both directions run on it."""
+    monkeypatch.setenv("SSM_LANES_PER_CHANNEL", "8")
+    monkeypatch.setenv("SSM_SCAN_WARPS", warps)
+    inp = synth.scan_inputs(2, 40, 300, 16, dtype, conv_width=4, bidirectional=True, seed=16)
+    for reverse in (False, True):
+        y, h = _run(inp, dtype, reverse=reverse, conv=True)
+        yo, ho = _oracle(inp, reverse=reverse, conv=True)
+        assert_close_out(host(y), yo, dtype, f"y ctas of {4 * int(warps)}")
+        state_close(host(h), ho, "final state")
+    y, h = _run(inp, dtype, conv=True, chunks=3)
+    yo, ho = _oracle(inp, conv=True)
+    assert_close_out(host(y), yo, dtype, "y two-pass")
+    state_close(host(h), ho, "final state two-pass")
+    y, hf, hr = _run(inp, dtype, conv=True, bidir=True)
+    yo, hfo, hro = _oracle(inp, conv=True, bidir=True)
+    assert_close_out(host(y), yo, dtype, "y bidirectional")
+    state_close(host(hf), hfo, "forward final state")
+    state_close(host(hr), hro, "reverse final state")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

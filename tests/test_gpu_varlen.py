@@ -54,12 +54,15 @@ LENGTHS = {
     "tile-aligned": [32, 32, 64, 96],
     "one-long": [700],
     "with-empty": [40, 0, 7, 0, 0, 60],
+    # sequences spanning several chunks (chunks with no start in them scan nothing) and
+    # starts off the tile grid
+    "spanning": [3, 500, 17, 1, 130],
 }
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("conv", [True, False])
-@pytest.mark.parametrize("chunks", [0, 3])
+@pytest.mark.parametrize("chunks", [0, 3, 7])
 @pytest.mark.parametrize("lengths", list(LENGTHS), ids=str)
 @pytest.mark.parametrize("dstate", [16, 5])
 def test_packed_sequences_match_oracle(dtype, conv, chunks, lengths, dstate):
@@ -77,10 +80,12 @@ def test_packed_sequences_match_oracle(dtype, conv, chunks, lengths, dstate):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_one_packed_sequence_equals_the_plain_call(dtype):
-    """A single packed sequence is the ordinary scan, bit for bit."""
+    """A single packed sequence is the ordinary scan, bit for bit (both in one pass: the
+    plain call would otherwise split this small grid into chunks with a carry, which
+    changes the rounding order)."""
     inp = synth.scan_inputs(1, 40, 333, 16, dtype, conv_width=4, seed=61)
-    a = _gpu(inp, dtype, _starts([333]), True)
-    b = _gpu(inp, dtype, None, True, packed=False)
+    a = _gpu(inp, dtype, _starts([333]), True, chunks=1)
+    b = _gpu(inp, dtype, None, True, chunks=1, packed=False)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
 
