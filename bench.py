@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--chunks", type=int, default=0, help="num_chunks passed to the scan (0 = auto)")
     ap.add_argument("--passes-per-step", type=int, default=0,
                     help="passes (one batch each) per bench step; 0 = enough for 25 ms")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (a smaller case of the same "
+                         "shape for profiler captures; the bench line names it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -168,7 +171,9 @@ def recorded_traffic(key, path=TRAFFIC_JSON):
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """nvidia-smi clock / throttle sampling while the timed region runs. start() returns
+    once the first sample has arrived (or after a few seconds), so that the sampler is
+    running when the timed region begins."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -176,8 +181,11 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.lines = []
+        self.reader = None
 
-    def start(self):
+    def start(self, wait_s: float = 3.0):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
@@ -185,18 +193,32 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        first = threading.Event()
 
-    def stop(self):
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append((time.perf_counter(), line))
+                first.set()
+        self.reader = threading.Thread(target=read, daemon=True)
+        self.reader.start()
+        first.wait(wait_s)
+
+    def stop(self, window=None):
+        """Median SM clock and throttle reasons over the samples that arrived inside
+        `window` (perf_counter seconds; all samples if none did), with their count."""
         if self.proc is None:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        if self.reader is not None:
+            self.reader.join(timeout=5)
         rows = []
-        for line in out.strip().splitlines():
+        inside = [ln for t, ln in self.lines if window and window[0] <= t <= window[1]]
+        for line in inside or [ln for _, ln in self.lines]:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -214,7 +236,8 @@ class ClockSampler:
                 if r[k].lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": rows[0]["max"],
-                "reasons": sorted(reasons), "samples": len(rows),
+                "reasons": sorted(reasons), "samples": len(self.lines),
+                "samples_under_load": len(inside),
                 "power_w_max": max(r["power"] for r in rows)}
 
 
@@ -691,9 +714,19 @@ def leave_ranks():
         dist.destroy_process_group()
 
 
+def workload_of(args):
+    """The named workload, with the sequence length overridden if asked."""
+    import dataclasses
+    w = synth.WORKLOADS[args.workload]
+    if args.seqlen and not w.name.startswith("decode"):
+        w = dataclasses.replace(w, seqlen=args.seqlen,
+                                name=f"{w.name} (seqlen overridden: {args.seqlen})")
+    return w
+
+
 def main():
     args = parse()
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -745,8 +778,8 @@ def main():
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.2)
     barrier()
+    w0 = time.perf_counter()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -756,7 +789,7 @@ def main():
         ev[2 * i + 1].record(stream)
     t1.record(stream)
     barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop((w0, time.perf_counter()))
     ms_total = t0.elapsed_time(t1)
     per_pass = [ev[2 * i].elapsed_time(ev[2 * i + 1]) / passes for i in range(args.steps)]
     ms_total = max_over_ranks(ms_total, device)
@@ -818,7 +851,7 @@ def main():
                "frac": sfu_ach / sfu_peak, "exp2_per_launch": exps,
                "peak_kind": (f"{N_SM} SMs x {SFU_EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
                              f"{sm_mhz:.0f} MHz (sampled SM clock)")}
-        traffic = recorded_traffic(args.workload)
+        traffic = None if args.seqlen else recorded_traffic(args.workload)
         if w.name.startswith("decode") or w.extra.get("conv_only"):
             roof = dict(bound="hbm", **{k: hbm[k] for k in ("achieved", "peak", "unit", "frac")},
                         traffic=traffic, peak_kind=hbm["peak_kind"],

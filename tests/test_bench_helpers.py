@@ -88,3 +88,29 @@ def test_default_workload_is_the_largest_single_gpu_config():
     w = W["long"]
     assert (w.batch, w.dim, w.seqlen, w.dstate, w.dtype, w.final_state) == (1, 5120, 65536, 16,
                                                                            "bf16", True)
+
+
+def test_clock_sampler_counts_the_samples_inside_the_timed_window(tmp_path, monkeypatch):
+    """A fake nvidia-smi prints one sample every 20 ms; start() returns once the first has
+    arrived, and stop() takes the median and the reasons over the window's samples."""
+    import os
+    import time
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\n"
+                    "while true; do\n"
+                    "  echo '0, 1965, 1965, 300.5, 0x0, Not Active, Not Active, Not Active, Active'\n"
+                    "  sleep 0.02\n"
+                    "done\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ['PATH']}")
+    s = bench.ClockSampler(0)
+    s.start()
+    assert s.lines, "start() returns after the first sample"
+    w0 = time.perf_counter()
+    time.sleep(0.3)
+    w1 = time.perf_counter()
+    time.sleep(0.1)
+    c = s.stop((w0, w1))
+    assert c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    assert 5 <= c["samples_under_load"] < c["samples"]
