@@ -17,8 +17,9 @@ namespace {
 template <typename T, int NP, int S, int KC, int SW>
 ScanVariant variant_of() {
     using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    using CfgV = ScanCfg<T, NP, S, KC, SW, true>;
     return ScanVariant{(int)sizeof(T), NP, S, KC, SW, Cfg::G, Cfg::NT, Cfg::TT, Cfg::HALO, Cfg::SMEM,
-                       Cfg::MIN_CTAS};
+                       Cfg::MIN_CTAS, CfgV::TT, CfgV::SMEM, CfgV::MIN_CTAS};
 }
 
 template <typename T, int W>

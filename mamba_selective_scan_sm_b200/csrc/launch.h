@@ -20,6 +20,9 @@ struct ScanVariant {
     int halo;           // conv history elements fetched with a tile
     int smem_bytes;     // dynamic shared memory per CTA
     int min_ctas;       // CTAs per SM the launch bounds are sized for
+    int tile_vl;        // the same three for the packed-sequence kernels
+    int smem_bytes_vl;
+    int min_ctas_vl;
 };
 
 // Returns false if (elem_size, np, s, kc, sw) has no compiled kernel.

@@ -54,6 +54,12 @@
 
 namespace ssm {
 
+// Bytes of one tile row in the splits of 8 lanes per channel with bf16 activations (the
+// narrow batches): 128 (64-step tiles, half the per-tile overhead) or 64.
+#ifndef SSM_NARROW_ROWB
+#define SSM_NARROW_ROWB 128
+#endif
+
 // Steps whose state-independent operands are prepared together (a divisor of 16).
 #ifndef SSM_SCAN_BATCH
 #define SSM_SCAN_BATCH 2
@@ -65,9 +71,12 @@ constexpr int kProBarrier = 1;                              // the producers' na
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <typename T, int NP, int S, int KC, int SW>
+// VLK: the packed-sequence kernels (their tile length may differ).
+template <typename T, int NP, int S, int KC, int SW, bool VLK = false>
 struct ScanCfg {
     static constexpr int SCAN_THREADS = 32 * SW; // SW recurrence warps
+    static constexpr bool ROWB_NARROW = sizeof(T) == 2 && S == 8 && NP * S == 16 && !VLK &&
+                                        SSM_NARROW_ROWB == 128;   // 64-step tiles
     static constexpr int G = SCAN_THREADS / S * KC;   // channels per CTA
     static constexpr int NT = SCAN_THREADS + kProThreads;   // threads per CTA
     // CTAs per SM the launch bounds ask for: three of 6 warps (96 registers per
@@ -75,12 +84,17 @@ struct ScanCfg {
     // two for d_state 64 / 128 (their B/C tiles take up to 127 KB of shared memory), one
     // of 10 warps with 8 scan warps
     static constexpr int MIN_CTAS =
-        SW == 8 ? 1 : NP * S > 16 ? 2 : (SW >= 3 || S == 2 || KC == 2 ? 3 : 5);
+        SW == 8 ? 1 : NP * S > 16 ? 2 : (SW >= 3 || S == 2 || KC == 2 ? 3 : ROWB_NARROW ? 4 : 5);
     static constexpr int NS = NP * S;            // padded state count
     static constexpr int ES = sizeof(T);
-    static constexpr int TT = 64 / ES;           // tile length: 32 (bf16) / 16 (fp32) steps
-    static constexpr int ROWB = TT * ES;         // bytes of one tile row (64)
-    static constexpr int SWZ = 3;                // TMA 64-B swizzle mask
+    // bytes of one tile row: 64 (32 bf16 / 16 fp32 steps); 128 (64 bf16 steps) in the
+    // narrow bf16 splits, where a CTA holds few channels and per-tile costs weigh most
+    // (not for packed sequences: measured slower there)
+    static constexpr int ROWB = ROWB_NARROW ? 128 : 64;
+    static constexpr int TT = ROWB / ES;         // tile length in steps
+    // TMA swizzle spanning one tile row (XOR of address bits [4, 4+w) with [7, 7+w)):
+    // 64-byte (w = 2) or 128-byte (w = 3)
+    static constexpr int SWZ = ROWB == 128 ? 7 : 3;
     static constexpr int HALO = 16 / ES;         // conv history, one 16-B TMA granule
     static constexpr int NSTAGE = 2;             // raw TMA stages
     static constexpr int NBUF = 2;               // staging buffers
@@ -119,7 +133,12 @@ struct ScanCfg {
     static_assert(BUF_E % 16 == 0 && BUF_BT % 16 == 0 && BUF % 16 == 0, "16-byte aligned parts");
     static_assert(NS <= 128, "at most 128 states");
     static_assert(KC == 1 || KC == 2, "one or two channels per lane");
-    static_assert(HALO + TT + 1 <= 64, "the packed-sequence window mask is 64 bits");
+    static_assert(HALO + TT + 1 <= 128, "the packed-sequence window mask is 128 bits");
+    static_assert(ROWB == 64 || ROWB == 128, "tile rows of 64 or 128 bytes");
+    // packed sequences: sequence starts at positions [l0 - HALO, l0 + TT] (Mask) and the
+    // tile's steps (Steps), one bit each
+    using Mask = std::conditional_t<(HALO + TT + 1 > 64), unsigned __int128, uint64_t>;
+    using Steps = std::conditional_t<(TT > 32), uint64_t, uint32_t>;
 };
 
 // Byte offset of logical (row, byte) in a swizzled [rows][ROWB] tile. TMA's 64-B
@@ -247,9 +266,10 @@ __device__ __noinline__ void put_conv_history(const ScanParams& p, uint8_t* raw_
 
 template <typename T, int NP, int S, int KC, int SW, bool USE_TMA, bool SUMMARY, bool VL,
           bool CL, int FEAT>
-__global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW>::NT, ScanCfg<T, NP, S, KC, SW>::MIN_CTAS)
+__global__ void __launch_bounds__(ScanCfg<T, NP, S, KC, SW, VL>::NT,
+                                  ScanCfg<T, NP, S, KC, SW, VL>::MIN_CTAS)
 scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
-    using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    using Cfg = ScanCfg<T, NP, S, KC, SW, VL>;
     constexpr int kScanWarps = SW, kScanThreads = Cfg::SCAN_THREADS, kCtaThreads = Cfg::NT;
     using E = Elem<T>;
     constexpr int G = Cfg::G, NS = Cfg::NS, TT = Cfg::TT, HALO = Cfg::HALO, R = Cfg::R;
@@ -470,13 +490,13 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 const int m = (a + z) >> 1;
                 if (p.cu[m] < lo) a = m + 1; else z = m;
             }
-            uint64_t wm = 0;
+            typename Cfg::Mask wm = 0;
             for (int i = a; i <= p.nseq && i < a + 2 * (TT + HALO + 2); ++i) {
                 const int s = p.cu[i];
                 if (s > l0 + TT) break;
-                if (s >= lo) wm |= 1ull << (s - lo);
+                if (s >= lo) wm |= typename Cfg::Mask(1) << (s - lo);
             }
-            *reinterpret_cast<uint64_t*>(buf + Cfg::BUF_META) = wm;
+            *reinterpret_cast<typename Cfg::Mask*>(buf + Cfg::BUF_META) = wm;
         };
 
         // Raw stage `st` of tile f -> staging buffer `buf`. Each producer thread owns a
@@ -487,8 +507,11 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             constexpr bool RV = decltype(rv_tag)::value;
             constexpr bool CONV = decltype(conv_tag)::value;
             constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte chunk
-            // steps per producer thread (at least one chunk; then not every thread has one)
-            constexpr int SEG = TT * G / kProThreads > EPC ? TT * G / kProThreads : EPC;
+            // steps per producer thread: whole 16-byte chunks, at least one (then not every
+            // thread has a segment)
+            constexpr int PER = TT * G / kProThreads;
+            constexpr int SEG = PER <= EPC ? EPC : (PER + EPC - 1) / EPC * EPC;
+            static_assert(TT % SEG == 0 && TT * G / SEG <= kProThreads, "segments tile the tile");
             [[maybe_unused]] constexpr int NSEG = TT * G / SEG;   // segments per tile
             constexpr int SUB = 2 * EPC < SEG ? 2 * EPC : SEG;  // steps per register window
             constexpr int NC = SUB / EPC;                     // dt / z chunks per window
@@ -544,13 +567,18 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             // P rows hold KC channels side by side: this channel's {delta, delta*u} slot
             uint8_t* prow_base = buf + Cfg::BUF_P + (r / KC) * Cfg::P_PITCH + (r % KC) * 8;
             // packed sequences: the conv of step ti reads no position before its start
-            const uint64_t wm = VL ? *reinterpret_cast<const uint64_t*>(buf + Cfg::BUF_META) : 0;
-            auto first_tap = [&](int ti) {            // first tap at or after the start
-                const uint32_t w4 = (uint32_t)(wm >> (HALO + ti - 3)) & 0xFu;
+            const typename Cfg::Mask wm =
+                VL ? *reinterpret_cast<const typename Cfg::Mask*>(buf + Cfg::BUF_META) : 0;
+            // first tap at or after the start for step s0 + i of the window, from the
+            // window's slice of the mask (bit m <-> position s0 - 3 + m; SUB + 3 <= 32)
+            static_assert(2 * EPC + 3 <= 32, "a register window's starts fit 32 bits");
+            auto first_tap = [&](uint32_t wwin, int i) {
+                const uint32_t w4 = (wwin >> i) & 0xFu;
                 return w4 ? 31 - __clz(w4) : 0;
             };
 #pragma unroll
             for (int s0 = t0; s0 < t0 + SEG; s0 += SUB) {
+                [[maybe_unused]] const uint32_t wwin = VL ? (uint32_t)(wm >> (HALO + s0 - 3)) : 0u;
                 // x window: row elements [s0, s0 + NXC*EPC). Forward rows start HALO steps
                 // before the tile (the conv history), reverse rows end HALO steps after it.
                 const uint4* xs = reinterpret_cast<const uint4*>(
@@ -596,7 +624,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     if constexpr (CONV) {
                         // forward: u_t = sum_k w_k x[t-3+k]; reverse: u_t = sum_k w_k x[t+3-k]
                         uint64_t acc = cb2;
-                        const int fa = VL ? first_tap(s0 + i) : 0, fb = VL ? first_tap(s0 + i + 1) : 0;
+                        const int fa = VL ? first_tap(wwin, i) : 0, fb = VL ? first_tap(wwin, i + 1) : 0;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int a = RV ? i + 3 - k : HALO + i - 3 + k;
@@ -872,8 +900,10 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
         const int l0 = RV ? L - i0 - TT : i0;
         const uint8_t* Prow = buf + Cfg::BUF_P + lg * Cfg::P_PITCH;
         // packed sequences: bit tt <-> step tt starts / ends a sequence
-        const uint64_t wm = VL ? *reinterpret_cast<const uint64_t*>(buf + Cfg::BUF_META) : 0;
-        const uint32_t starts = (uint32_t)(wm >> HALO), ends = (uint32_t)(wm >> (HALO + 1));
+        const typename Cfg::Mask wm =
+            VL ? *reinterpret_cast<const typename Cfg::Mask*>(buf + Cfg::BUF_META) : 0;
+        using Steps = typename Cfg::Steps;
+        const Steps starts = (Steps)(wm >> HALO), ends = (Steps)(wm >> (HALO + 1));
         // a sequence ended at step tt: its final state (the sequence is the last one whose
         // start is <= l0 + tt; empty sequences share their successor's start)
         auto seq_end = [&](int tt) {

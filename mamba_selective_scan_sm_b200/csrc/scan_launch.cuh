@@ -10,7 +10,7 @@ namespace {
 template <typename T, int NP, int S, int KC, int SW, bool TMA, bool SUM, bool VL, bool CL,
           int FEAT>
 cudaError_t launch_one(const ScanMaps& maps, const ScanParams& p, dim3 grid, cudaStream_t st) {
-    using Cfg = ScanCfg<T, NP, S, KC, SW>;
+    using Cfg = ScanCfg<T, NP, S, KC, SW, VL>;
     auto* k = scan_fwd_kernel<T, NP, S, KC, SW, TMA, SUM, VL, CL, FEAT>;
     static const cudaError_t attr =
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);

@@ -101,7 +101,6 @@ struct DecodeParams {
     int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
     int stream;         // streaming variant: dstate 16, dim % 128 == 0, 16-byte aligned bases
     int head_dim;       // A one scalar per head (A[d / head_dim]); 0: A is (dim, dstate)
-    int vec_bc;         // B_t, C_t rows in 16-byte chunks: dstate % 16 == 0, 16-byte bases
 };
 
 }  // namespace ssm

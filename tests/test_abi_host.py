@@ -166,10 +166,14 @@ def test_workspace_size_query(lib):
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 0                               # single pass, one direction
     # automatic: 2 x 64 channels in 8-channel CTAs fill few of the 148 SMs' slots, so the
-    # sequence (4 tiles of 32 steps) is split into as many chunks as it has tiles
+    # sequence (2 tiles of 64 bf16 steps in these narrow splits) is split into as many
+    # chunks as it has tiles: one summary chunk
     a = _args()
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
-    assert n.value == 3 * 2 * 64 * 16 * 8
+    assert n.value == 1 * 2 * 64 * 16 * 8
+    a = _args(dtype=0)                                # fp32: 8 tiles of 16 steps
+    assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 7 * 2 * 64 * 16 * 8
     a = _args(dim=9472 * 2)                           # enough channels: one pass
     assert lib.ssm_selective_scan_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 0
