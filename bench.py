@@ -396,13 +396,15 @@ class ScanWorkload:
 class ConvWorkload:
     """The standalone causal conv1d + SiLU (ssm_causal_conv1d_fwd) on the m130 shape.
 
-    One step's 100 MB (x read, y written) would fit the 126 MB L2, so steps rotate over
-    SETS independent input/output pairs: a step's tensors were last touched SETS - 1
-    steps earlier, with ~200 MB of other traffic in between. The launch (~21 us) is
-    shorter than the binding's host-side call, so each set's launch is captured once in
-    a CUDA graph and a step replays it (the end-to-end leg calls the binding itself)."""
+    One launch's 100 MB (x read, y written) would fit the 126 MB L2, so launches rotate
+    over SETS independent input/output pairs: a launch's tensors were last touched SETS - 1
+    launches earlier, with ~200 MB of other traffic in between. A launch (~21 us) is
+    shorter than the binding's host-side call and than the gap between two graph
+    replays, so one CUDA graph holds REP launches cycling over the sets and a pass replays
+    it: REP batches per pass (the end-to-end leg calls the binding itself)."""
 
     SETS = 3
+    REP = 30
 
     def __init__(self, w, device):
         import torch
@@ -418,27 +420,23 @@ class ConvWorkload:
         self.cw = torch.from_numpy(inp["conv_w"]).to(device)
         self.cb = torch.from_numpy(inp["conv_b"]).to(device)
         self.k = 0
-        self.launches_per_pass = 1
+        self.launches_per_pass = self.REP
         self.h = None
         self.launch(0)                                  # load the kernel outside the capture
         torch.cuda.synchronize()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
-        self.graphs = []
-        for i in range(self.SETS):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
-                self.launch(i)
-            self.graphs.append(g)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side), torch.cuda.graph(self.graph, stream=side):
+            for i in range(self.REP):
+                self.launch(i % self.SETS)
         torch.cuda.current_stream().wait_stream(side)
 
     def launch(self, i):
         self.ssm.ssm_causal_conv1d_fwd(self.xs[i], self.cw, self.cb, True, out=self.outs[i])
 
     def unit(self):
-        i = self.k % self.SETS
-        self.k += 1
-        self.graphs[i].replay()
+        self.graph.replay()
 
     def e2e_setup(self):
         self.h = self.x.cpu().pin_memory()
@@ -454,9 +452,10 @@ class ConvWorkload:
         self.hout.copy_(self.outs[i], non_blocking=True)
 
     e2e_pipelined = None
+    batches_per_unit = REP                            # e2e_serial moves one batch
 
     def elems(self):
-        return self.w.batch * self.w.dim * self.w.seqlen
+        return self.REP * self.w.batch * self.w.dim * self.w.seqlen
 
 
 class DecodeWorkload:
@@ -652,8 +651,10 @@ def config_of(w, args, passes=1):
         c["launch"] = f"one CUDA graph of {w.steps} token launches per step"
     ab = algorithmic_bytes(w)
     if w.extra.get("conv_only"):
-        c["l2"] = (f"steps rotate over {ConvWorkload.SETS} input/output pairs "
+        c["l2"] = (f"launches rotate over {ConvWorkload.SETS} input/output pairs "
                    f"({ConvWorkload.SETS * ab / 1e6:.0f} MB > 126 MB L2)")
+        c["launch"] = (f"one CUDA graph of {ConvWorkload.REP} launches per pass, "
+                       f"each one batch of the shape above")
     elif w.name.startswith("decode"):
         es = 2 if w.dtype == "bf16" else 4
         layer_mb = w.batch * w.dim * (w.dstate * 4 + w.conv_width * es) / 1e6   # SSM + conv state
@@ -817,28 +818,30 @@ def main():
 
         k = max(3, min(args.steps, 10))
         ms_serial = timed(wl.e2e_serial, k)        # per batch
-        e2e = {"unit": "elems/s", "h2d_bytes_per_step": wl.h2d * passes,
-               "d2h_bytes_per_step": wl.d2h * passes}
-        serial = {"value": job_throughput(wl.elems(), world, ms_serial), "ms_per_batch": ms_serial,
+        bpu = getattr(wl, "batches_per_unit", 1)   # batches one pass of the device leg holds
+        batch_elems = wl.elems() // bpu
+        e2e = {"unit": "elems/s", "h2d_bytes_per_step": wl.h2d * passes * bpu,
+               "d2h_bytes_per_step": wl.d2h * passes * bpu}
+        serial = {"value": job_throughput(batch_elems, world, ms_serial), "ms_per_batch": ms_serial,
                   "how": "upload, scan and read-back of one batch back to back on one stream"}
         if wl.e2e_pipelined is not None:
             nb = max(4, k)
             ms_pipe = timed(lambda: wl.e2e_pipelined(nb), 1) / nb
-            e2e.update(value=job_throughput(wl.elems(), world, ms_pipe), ms_per_step=ms_pipe * passes,
+            e2e.update(value=job_throughput(batch_elems, world, ms_pipe), ms_per_step=ms_pipe * passes * bpu,
                        ms_per_batch=ms_pipe,
                        how=(f"{nb} batches: uploads on one copy stream, scans on the compute "
                             "stream, read-backs on a second copy stream, two device input sets"),
                        serial=serial)
         else:
-            e2e.update(value=serial["value"], ms_per_step=ms_serial * passes,
+            e2e.update(value=serial["value"], ms_per_step=ms_serial * passes * bpu,
                        ms_per_batch=ms_serial, how=serial["how"])
 
     if rank == 0:
         hbm_peak, peak_kind = measured_peaks()
         ab = algorithmic_bytes(w)
-        # a decode pass is a graph of back-to-back launches of one kernel
-        mean_launch_ms = statistics.mean(per_pass) / (wl.launches_per_pass
-                                                      if w.name.startswith("decode") else 1)
+        # a decode or conv pass is a graph of back-to-back launches of one kernel
+        mean_launch_ms = statistics.mean(per_pass) / (
+            wl.launches_per_pass if (w.name.startswith("decode") or w.extra.get("conv_only")) else 1)
         achieved = ab / (mean_launch_ms * 1e-3) / 1e9
         sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
         exps = exp_count(w) / (w.steps if w.steps else 1) if w.name.startswith("decode") else exp_count(w)

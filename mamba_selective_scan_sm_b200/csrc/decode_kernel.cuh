@@ -569,4 +569,209 @@ __global__ void __launch_bounds__(256) decode_warp_kernel(const DecodeParams p) 
     }
 }
 
+// Streaming decode for d_state 32, 64 or 128 (LPC = d_state / 16 lanes per channel,
+// 16 states per lane) with A per head or per (channel, state). A tile is one batch row's
+// R = 256 / LPC consecutive channels: their fp32 state (R * d_state * 4 = 16 KB, one
+// contiguous range), conv state, x, dt, z, and the batch row's B_t and C_t. Tiles stream
+// through a kStreamStages-deep ring of 1-D bulk copies and leave with bulk stores, as in
+// decode_stream_kernel; the grid is one wave of CTAs, each a contiguous range of the
+// (channel group, batch row) tiles taken group-major, so the per-channel parameters stay
+// in registers until the range crosses into the next group. Lane q of a channel holds,
+// for g = 0..3, the four states n = 4 * (LPC * ch + q) .. + 3 of chunk ch = (g + c) & 3:
+// the eight lanes of a quarter-warp then read 128 distinct bytes of shared memory. With
+// A per head the decay exp(delta * A_h) is one exp per channel for all its states.
+// Requires dim % R == 0, 16-byte aligned bases (checked on the host).
+template <typename T, int LPC>
+struct WideTile {
+    static constexpr int ES = sizeof(T);
+    static constexpr int R = 256 / LPC;                               // channels per tile
+    static constexpr int N = 16 * LPC;                                // states per channel
+    static constexpr int STATE = 0;                                   // [R][N] fp32
+    static constexpr int CONV = STATE + R * N * 4;                    // [R][W] T, W <= 4
+    static constexpr int X = CONV + R * 4 * ES;
+    static constexpr int DT = X + R * ES;
+    static constexpr int Z = DT + R * ES;
+    static constexpr int Y = Z + R * ES;                              // output
+    static constexpr int BT = Y + R * ES;                             // [N] T
+    static constexpr int CT = BT + N * ES;
+    static constexpr int BYTES = (CT + N * ES + 127) / 128 * 128;
+    static_assert(CONV % 16 == 0 && X % 16 == 0 && DT % 16 == 0 && Z % 16 == 0 && Y % 16 == 0 &&
+                  BT % 16 == 0 && CT % 16 == 0, "bulk copies need 16-byte aligned parts");
+};
+
+template <typename T, int LPC>
+__global__ void __launch_bounds__(256, 3) decode_wide_stream_kernel(const DecodeParams p) {
+    using E = Elem<T>;
+    using Tl = WideTile<T, LPC>;
+    constexpr int R = Tl::R, N = Tl::N, ES = Tl::ES;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ uint64_t full[kStreamStages];
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int c = tid / LPC, q = tid % LPC;           // channel within the tile, lane in it
+    const int rot = c & 3;
+    const int W = p.conv_w ? p.conv_width : 0;
+    const bool gate = p.z != nullptr, heads = p.head_dim != 0;
+    const int64_t batch = p.rows / p.dim;
+    const int64_t ntot = batch * (p.dim / R);
+    const int64_t tfirst = ntot * blockIdx.x / gridDim.x;
+    const int ntiles = (int)(ntot * (blockIdx.x + 1) / gridDim.x - tfirst);
+    if (ntiles == 0) return;                          // uniform over the CTA
+    const int g0 = (int)(tfirst / batch);             // the range's first (group, batch row)
+    const int64_t b0 = tfirst - (int64_t)g0 * batch;
+    const uint32_t cs_bytes = R * W * ES, v_bytes = R * ES;
+    const uint32_t tile_bytes = R * N * 4 + cs_bytes + v_bytes * (gate ? 3 : 2) + 2 * N * ES;
+
+    auto stage = [&](int i) { return dsm + (i % kStreamStages) * Tl::BYTES; };
+    int64_t ib = b0;                                  // the next tile to issue (thread 0)
+    int ig = g0;
+    auto issue = [&](int i) {
+        uint8_t* s = stage(i);
+        const int64_t r0 = ib * p.dim + (int64_t)ig * R;
+        uint64_t* bar = &full[i % kStreamStages];
+        mbar_arrive_expect_tx(bar, tile_bytes);
+        bulk_load(s + Tl::STATE, p.state + r0 * N, R * N * 4, bar);
+        if (W) bulk_load(s + Tl::CONV, static_cast<const T*>(p.conv_state) + r0 * W, cs_bytes, bar);
+        bulk_load(s + Tl::X, static_cast<const T*>(p.x) + r0, v_bytes, bar);
+        bulk_load(s + Tl::DT, static_cast<const T*>(p.dt) + r0, v_bytes, bar);
+        if (gate) bulk_load(s + Tl::Z, static_cast<const T*>(p.z) + r0, v_bytes, bar);
+        bulk_load(s + Tl::BT, static_cast<const T*>(p.Bt) + ib * N, N * ES, bar);
+        bulk_load(s + Tl::CT, static_cast<const T*>(p.Ct) + ib * N, N * ES, bar);
+        if (++ib == batch) { ib = 0; ++ig; }
+    };
+
+    int issued = 0;
+    if (tid == 0) {
+        for (int k = 0; k < kStreamStages; ++k) mbar_init(&full[k], 1);
+        fence_mbar_init();
+        for (; issued < min(kStreamStages, ntiles); ++issued) issue(issued);
+    }
+
+    // the channel's parameters, reloaded when the range enters the next channel group
+    uint64_t a2[8];                                   // A * log2(e) as pairs, chunk-rotated
+    float ah = 0.f, w4[4], cb = 0.f, dbias = 0.f, Dv = 0.f;
+    auto load_params = [&](int grp) {
+        const int d = grp * R + c;
+        if (heads) {
+            ah = __ldg(p.A + d / p.head_dim) * kLog2e;
+        } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const int n0 = 4 * (LPC * ((g + rot) & 3) + q);
+                const float4 a4 = __ldg(reinterpret_cast<const float4*>(p.A + (int64_t)d * N + n0));
+                a2[2 * g] = pk2(a4.x * kLog2e, a4.y * kLog2e);
+                a2[2 * g + 1] = pk2(a4.z * kLog2e, a4.w * kLog2e);
+            }
+        }
+        // taps right-aligned: w4[3] meets the newest input
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int kk = k - (4 - W);
+            w4[k] = kk >= 0 ? __ldg(p.conv_w + (int64_t)d * W + kk) : 0.f;
+        }
+        cb = W && p.conv_b ? __ldg(p.conv_b + d) : 0.f;
+        dbias = p.dt_bias ? __ldg(p.dt_bias + d) : 0.f;
+        Dv = p.D ? __ldg(p.D + d) : 0.f;
+    };
+    int grp = g0;
+    load_params(grp);
+    int64_t b = b0;
+
+    auto wait_tile = [&](int i) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(&full[i % kStreamStages], (i / kStreamStages) & 1);
+        return ok;
+    };
+    auto drain = [&](int from) {                      // thread 0, on the way out
+        if (tid != 0) return;
+        for (int k = from; k < issued; ++k)
+            mbar_wait_bounded(&full[k % kStreamStages], (k / kStreamStages) & 1);
+        bulk_wait_read();
+    };
+
+    __syncthreads();                                  // barrier init before any wait
+    if (__syncthreads_or(!wait_tile(0))) { drain(0); return; }
+    for (int i = 0; i < ntiles; ++i) {
+        uint8_t* s = stage(i);
+        mbar_try_wait(&full[i % kStreamStages], (i / kStreamStages) & 1);
+        const float xt = E::to_f(reinterpret_cast<const T*>(s + Tl::X)[c]);
+        T* scv = reinterpret_cast<T*>(s + Tl::CONV) + c * W;
+        float xc = xt;
+        T win[3];                                     // conv_state[1 .. W-1], oldest first
+        if (W) {
+            float acc = fmaf(w4[3], xt, cb);
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const int kk = k - (4 - W);           // window slot k + 1 - (4 - W) < W - 1
+                win[k] = kk >= 0 ? scv[kk + 1] : E::from_f(0.f);
+                if (kk >= 0) acc = fmaf(w4[k], E::to_f(win[k]), acc);
+            }
+            xc = silu(acc);
+        }
+        float dl = E::to_f(reinterpret_cast<const T*>(s + Tl::DT)[c]) + dbias;
+        if (p.softplus) dl = softplus(dl);
+        const uint64_t dd = pk2(dl, dl), uu = pk2(dl * xc, dl * xc);
+        const float dAh = heads ? ex2(dl * ah) : 0.f;
+        const uint64_t dA2h = pk2(dAh, dAh);
+        float* hrow = reinterpret_cast<float*>(s + Tl::STATE) + c * N;
+        uint64_t acc2 = pk2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int n0 = 4 * (LPC * ((g + rot) & 3) + q);
+            float bv[4], cv[4];
+            load4<T>(s + Tl::BT + n0 * ES, bv);
+            load4<T>(s + Tl::CT + n0 * ES, cv);
+            float4* hp = reinterpret_cast<float4*>(hrow + n0);
+            const float4 h4 = *hp;
+            uint64_t h[2] = {pk2(h4.x, h4.y), pk2(h4.z, h4.w)};
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                uint64_t dA = dA2h;
+                if (!heads) {
+                    const uint64_t x = mul2(dd, a2[2 * g + k]);
+                    dA = pk2(ex2(lo2(x)), ex2(hi2(x)));
+                }
+                h[k] = fma2(dA, h[k], mul2(uu, pk2(bv[2 * k], bv[2 * k + 1])));
+                acc2 = fma2(pk2(cv[2 * k], cv[2 * k + 1]), h[k], acc2);
+            }
+            *hp = make_float4(lo2(h[0]), hi2(h[0]), lo2(h[1]), hi2(h[1]));
+        }
+        float y = lo2(acc2) + hi2(acc2);
+#pragma unroll
+        for (int m = LPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+        __syncwarp();                                 // the channel's lanes have read its window
+        if (q == 0) {
+            y = fmaf(Dv, xc, y);
+            if (gate) y *= silu(E::to_f(reinterpret_cast<const T*>(s + Tl::Z)[c]));
+            reinterpret_cast<T*>(s + Tl::Y)[c] = E::from_f(y);
+            if (W) {                                  // shift the window, append x_t
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    if (k - (4 - W) >= 0) scv[k - (4 - W)] = win[k];
+                scv[W - 1] = reinterpret_cast<const T*>(s + Tl::X)[c];
+            }
+        }
+        fence_proxy_async_smem();                     // generic writes -> bulk-store reads
+        const bool ok = i + 1 < ntiles ? wait_tile(i + 1) : true;
+        if (__syncthreads_or(!ok)) { drain(i + 1); return; }
+        if (tid == 0) {
+            const int64_t r0 = b * p.dim + (int64_t)grp * R;
+            bulk_store(p.state + r0 * N, s + Tl::STATE, R * N * 4);
+            if (W) bulk_store(static_cast<T*>(p.conv_state) + r0 * W, s + Tl::CONV, cs_bytes);
+            bulk_store(static_cast<T*>(p.out) + r0, s + Tl::Y, v_bytes);
+            bulk_commit();
+            // the stage of tile i - 1 is free once its stores have read it
+            if (i >= 1 && issued < ntiles) {
+                asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                issue(issued++);
+            }
+        }
+        if (++b == batch && i + 1 < ntiles) {         // the next tile starts the next group
+            b = 0;
+            load_params(++grp);
+        }
+    }
+    if (tid == 0) bulk_wait_read();
+}
+
 }  // namespace ssm

@@ -33,6 +33,29 @@ cudaError_t launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <typename T, int LPC>
+cudaError_t launch_wide_stream(const DecodeParams& p, cudaStream_t st) {
+    constexpr int smem = kStreamStages * WideTile<T, LPC>::BYTES;
+    auto* k = decode_wide_stream_kernel<T, LPC>;
+    static int per_sm = 0;                            // resident CTAs per SM
+    if (per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    }
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // one wave: every CTA resident at once, each a contiguous range of tiles
+    const int64_t tiles = p.rows / WideTile<T, LPC>::R;
+    const int64_t grid = tiles < (int64_t)sms * per_sm ? tiles : (int64_t)sms * per_sm;
+    k<<<(unsigned)grid, 256, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool scan_variant(int es, int np, int s, int kc, int sw, ScanVariant* v) {
@@ -124,6 +147,19 @@ cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_
 }
 
 cudaError_t launch_decode_warp(int es, const DecodeParams& p, cudaStream_t st) {
+    if (p.stream) {                                   // d_state 32, 64, 128 in channel groups
+        const int lpc = p.dstate / 16;
+#define SSM_WIDE_LPC(T_, L_) \
+        if (lpc == L_) return launch_wide_stream<T_, L_>(p, st);
+        if (es == 2) {
+            SSM_WIDE_LPC(__nv_bfloat16, 2) SSM_WIDE_LPC(__nv_bfloat16, 4)
+            SSM_WIDE_LPC(__nv_bfloat16, 8)
+        } else {
+            SSM_WIDE_LPC(float, 2) SSM_WIDE_LPC(float, 4) SSM_WIDE_LPC(float, 8)
+        }
+#undef SSM_WIDE_LPC
+        return cudaErrorInvalidValue;
+    }
     // lanes per row: 16 states per lane
     const int lpr = p.dstate <= 16 ? 1 : p.dstate <= 32 ? 2 : p.dstate <= 64 ? 4 : 8;
     const int per_block = 8 * (32 / lpr);                       // channels per 8-warp block

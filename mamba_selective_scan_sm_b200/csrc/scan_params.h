@@ -99,7 +99,9 @@ struct DecodeParams {
     int dim, dstate, conv_width, softplus;
     int vec;            // dstate == 16 and state / A rows 16-byte aligned
     int bulk;           // bulk-copy variant: rows % 64 == 0, 16-byte aligned bases
-    int stream;         // streaming variant: dstate 16, dim % 128 == 0, 16-byte aligned bases
+    int stream;         // streaming variant (bulk-copy ring): dstate 16 in 128-channel groups,
+                        // or dstate 32 / 64 / 128 in 4096 / dstate channel groups; 16-byte
+                        // aligned bases
     int head_dim;       // A one scalar per head (A[d / head_dim]); 0: A is (dim, dstate)
 };
 

@@ -721,6 +721,18 @@ ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* a, ssm_strea
     p.softplus = a->dt_softplus ? 1 : 0;
     p.vec = a->dstate % 4 == 0 && aligned(a->state, 16);
     p.head_dim = a->a_heads > 0 ? (int)(a->dim / a->a_heads) : 0;
+    // Streaming (the default where it applies): d_state 32, 64 or 128, channel groups of
+    // 4096 / d_state, 16-byte aligned bases for its bulk copies. Else plain loads, one
+    // warp per 32 / lanes-per-row rows. SSM_DECODE_KERNEL = plain restricts the choice.
+    const int64_t group = a->dstate > 0 ? 4096 / a->dstate : 0;
+    const char* want = getenv("SSM_DECODE_KERNEL");
+    const bool plain = want && strcmp(want, "plain") == 0;
+    p.stream = !plain && (a->dstate == 32 || a->dstate == 64 || a->dstate == 128) &&
+               a->dim % group == 0 && aligned(a->state, 16) && aligned(a->x, 16) &&
+               aligned(a->dt, 16) && aligned(a->out, 16) && aligned(a->B_t, 16) &&
+               aligned(a->C_t, 16) && (!a->z || aligned(a->z, 16)) &&
+               (!a->conv_weight || aligned(a->conv_state, 16)) &&
+               (a->a_heads > 0 || aligned(a->A, 16));
     cudaError_t e = ssm::launch_decode_warp(es, p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state update launch");
     return ok();

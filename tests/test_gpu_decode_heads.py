@@ -1,8 +1,12 @@
 """GPU parity of the decode step with d_state up to 128 and with A one scalar per head
 (ssm_selective_state_update_ex, reached through the binding when A is 1-D or d_state is
 above 16) against the CPU oracle, over several successive steps: ragged row counts,
-d_state not a multiple of 4, both dtypes, with and without the conv and the gate; and
-decode steps against the scan of the same sequence on the GPU."""
+d_state not a multiple of 4, both dtypes, with and without the conv and the gate; the
+streaming kernel (d_state 32, 64, 128 in whole channel groups) over conv widths, short and
+long per-CTA tile ranges and ranges that cross channel groups, beside the plain kernel;
+and decode steps against the scan of the same sequence on the GPU."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -84,3 +88,42 @@ def test_decode_steps_equal_scan_on_gpu(dtype, N, heads):
     yd = np.stack([host(v) for v in ys], axis=-1)
     assert_close_out(yd, host(y), dtype, "decode vs scan", ulp=False)
     state_close(host(st), host(h), "decode vs scan state")
+
+
+def _check(inp, dtype, steps, conv, gate):
+    # a nonzero conv bias, so that a dropped or misplaced bias shows
+    inp["conv_b"] = np.random.default_rng(7).normal(0, 0.5, inp["conv_b"].shape).astype(np.float32)
+    yg, sg, cg = _gpu(inp, dtype, steps, conv, gate)
+    yo, so, co = _ref(inp, steps, conv, gate)
+    for s in range(steps):
+        assert_close_out(yg[s], yo[s], dtype, f"y step {s}")
+    state_close(sg, so, "state")
+    if conv:
+        np.testing.assert_array_equal(cg, co)
+
+
+# (d_state, heads, dim): dim a whole number of 4096 / d_state channel groups
+STREAM_SHAPES = [(128, 4, 96), (128, 0, 64), (64, 3, 192), (64, 0, 128), (32, 2, 256),
+                 (32, 0, 128)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,heads,D", STREAM_SHAPES)
+@pytest.mark.parametrize("width,gate", [(4, True), (3, False), (2, True), (1, False), (0, True)])
+@pytest.mark.parametrize("kernel", ["", "plain"])
+def test_streaming_decode_shapes(dtype, N, heads, D, width, gate, kernel, monkeypatch):
+    """The streaming kernel (default for these shapes) and the plain one, against the
+    oracle: one tile per CTA (B * D / group tiles below one wave)."""
+    monkeypatch.setenv("SSM_DECODE_KERNEL", kernel)
+    inp = synth.decode_inputs(5, D, N, 3, max(width, 1), dtype, seed=101, a_heads=heads)
+    _check(inp, dtype, 3, width > 0, gate)
+
+
+@pytest.mark.parametrize("dtype,N,heads,B,D", [("bf16", 128, 4, 1000, 96), ("f32", 128, 0, 700, 64),
+                                              ("f32", 32, 2, 600, 256), ("bf16", 64, 0, 450, 192)])
+def test_streaming_decode_long_ranges(dtype, N, heads, B, D):
+    """More tiles than one wave of CTAs: each CTA walks a range of several tiles through
+    the copy ring, and ranges cross from one channel group into the next."""
+    assert os.environ.get("SSM_DECODE_KERNEL", "") in ("", "stream")
+    inp = synth.decode_inputs(B, D, N, 2, 4, dtype, seed=102, a_heads=heads)
+    _check(inp, dtype, 2, True, True)
