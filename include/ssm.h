@@ -263,9 +263,12 @@ typedef struct {
 
 /* The decode step of ssm_selective_state_update, for d_state up to SSM_MAX_SCAN_DSTATE
  * and A per head (the step method of the scan's per-head form). With d_state <= 16 and
- * a_heads = 0 it runs the same kernels as ssm_selective_state_update. Errors as there;
- * SSM_ERR_BAD_SHAPE also for a_heads < 0 or not dividing dim; SSM_ERR_ALIAS also when
- * conv_state overlaps state. */
+ * a_heads = 0 it runs the same kernels as ssm_selective_state_update. With d_state 32, 64
+ * or 128, dim a multiple of 4096 / d_state and 16-byte aligned state, conv_state, x, dt,
+ * z, out, B_t, C_t (and A when it is per state), the step streams groups of channels
+ * through shared memory with bulk copies; otherwise it uses plain loads. Same results
+ * either way, within rounding. Errors as there; SSM_ERR_BAD_SHAPE also for a_heads < 0
+ * or not dividing dim; SSM_ERR_ALIAS also when conv_state overlaps state. */
 SSM_API ssm_status_t ssm_selective_state_update_ex(const ssm_update_args_t* args,
                                                    ssm_stream_t stream);
 

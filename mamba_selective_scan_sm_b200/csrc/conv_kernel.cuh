@@ -5,7 +5,7 @@
 // one read and one write per element, so it is HBM-bound: each thread produces 32
 // bytes of consecutive outputs from two aligned 16-byte loads plus the 16-byte chunk
 // before them (for the 3 preceding inputs; the neighbouring thread's chunk, an L1
-// hit), with the taps, the conv and the SiLU on packed fp32 pairs.
+// hit), with the taps as scalar FMAs and the SiLU on packed fp32 pairs.
 #pragma once
 
 #include "device_common.cuh"
@@ -14,11 +14,16 @@
 namespace ssm {
 
 
+constexpr int kConvChunks = 2;                            // 16-byte output chunks per thread
+constexpr int kConvThreads = 256 / kConvChunks;
+
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvParams p) {
     using E = Elem<T>;
+    constexpr int CH = kConvChunks;
     constexpr int EPC = 16 / (int)sizeof(T);              // elements per 16-byte chunk
-    constexpr int V = 2 * EPC;                            // outputs per thread (32 bytes)
+    constexpr int V = CH * EPC;                           // outputs per thread
+    grid_dependency_sync();                               // launched as a dependent
     const int L = p.seqlen;
     // grid: x = runs of V outputs along the row, y = row (b, d) in slabs of 65535
     const int t0 = (int)(blockIdx.x * blockDim.x + threadIdx.x) * V;
@@ -41,23 +46,33 @@ __global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
     if (VEC && t0 + V <= L) {
         // x[t0 - EPC .. t0 + V): the chunk before (for the 3 previous inputs) and the
         // thread's two chunks; position t0 - 3 + m is window element EPC - 3 + m
-        const uint4 win[3] = {t0 >= EPC ? *reinterpret_cast<const uint4*>(xr + t0 - EPC)
-                                        : make_uint4(0, 0, 0, 0),
-                              *reinterpret_cast<const uint4*>(xr + t0),
-                              *reinterpret_cast<const uint4*>(xr + t0 + EPC)};
+        uint4 win[CH + 1];
+        win[0] = t0 >= EPC ? *reinterpret_cast<const uint4*>(xr + t0 - EPC) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) win[c + 1] = *reinterpret_cast<const uint4*>(xr + t0 + c * EPC);
+        // the window widened once; the taps as scalar FMAs on it (a packed pair of
+        // overlapping window elements would need register moves for every tap)
+        float xf[(CH + 1) * EPC];
+#pragma unroll
+        for (int m = EPC - 3; m < (CH + 1) * EPC; ++m) xf[m] = chunk_elem<T>(win, m);
+        float wk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) wk[k] = lo2(w2[k]);
         uint32_t ob[V / 2];                               // bf16 pairs, or fp32 bits
         float of[V];
 #pragma unroll
         for (int i = 0; i < V; i += 2) {                  // outputs t0 + i, t0 + i + 1
-            uint64_t acc = pk2(bias, bias);
+            float a0 = bias, a1 = bias;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                acc = fma2(w2[k], pk2(chunk_elem<T>(win, EPC - 3 + i + k),
-                                      chunk_elem<T>(win, EPC - 2 + i + k)), acc);
-            // SiLU with one SFU op per output (the reciprocal on the FMA pipe): 2 Newton
-            // steps leave 1.2e-5 relative error, far below a bf16 output's rounding;
-            // fp32 outputs take 3 (1.5e-10)
-            if (p.silu) acc = sizeof(T) == 2 ? silu2_fma<2>(acc) : silu2_fma<3>(acc);
+            for (int k = 0; k < 4; ++k) {
+                a0 = fmaf(wk[k], xf[EPC - 3 + i + k], a0);
+                a1 = fmaf(wk[k], xf[EPC - 2 + i + k], a1);
+            }
+            uint64_t acc = pk2(a0, a1);
+            // SiLU with the exp and the reciprocal on the SFU: the kernel is issue-bound
+            // before it is SFU-bound, and the FMA-pipe reciprocal (silu2_fma) takes
+            // seven instructions per output against four
+            if (p.silu) acc = silu2(acc);
             const float2 y = upk2(acc);
             if constexpr (sizeof(T) == 2) {
                 __nv_bfloat162 t2 = __floats2bfloat162_rn(y.x, y.y);
@@ -67,12 +82,14 @@ __global__ void __launch_bounds__(128) conv1d_kernel(const ConvParams p) {
                 of[i + 1] = y.y;
             }
         }
-        if constexpr (sizeof(T) == 2) {
-            *reinterpret_cast<uint4*>(yr + t0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-            *reinterpret_cast<uint4*>(yr + t0 + EPC) = make_uint4(ob[4], ob[5], ob[6], ob[7]);
-        } else {
-            *reinterpret_cast<float4*>(yr + t0) = make_float4(of[0], of[1], of[2], of[3]);
-            *reinterpret_cast<float4*>(yr + t0 + 4) = make_float4(of[4], of[5], of[6], of[7]);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            if constexpr (sizeof(T) == 2)
+                *reinterpret_cast<uint4*>(yr + t0 + c * EPC) =
+                    make_uint4(ob[4 * c], ob[4 * c + 1], ob[4 * c + 2], ob[4 * c + 3]);
+            else
+                *reinterpret_cast<float4*>(yr + t0 + c * EPC) =
+                    make_float4(of[4 * c], of[4 * c + 1], of[4 * c + 2], of[4 * c + 3]);
         }
         return;
     }

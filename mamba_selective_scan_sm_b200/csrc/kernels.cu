@@ -93,20 +93,19 @@ cudaError_t launch_conv_tail(int es, const ConvTailParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_conv(int es, bool vec, const ConvParams& p, cudaStream_t st) {
-    const int64_t per_row = (p.seqlen + 32 / es - 1) / (32 / es);   // 32 bytes per thread
-    const unsigned bx = (unsigned)((per_row + 127) / 128);
+    const int v = kConvChunks * 16 / es;                            // outputs per thread
+    const int64_t per_row = (p.seqlen + v - 1) / v;
+    const unsigned bx = (unsigned)((per_row + kConvThreads - 1) / kConvThreads);
     const unsigned by = (unsigned)(p.rows < 65535 ? p.rows : 65535);
     const int64_t bz = (p.rows + 65534) / 65535;
     if (bz > 65535) return cudaErrorInvalidConfiguration;
     const dim3 grid(bx, by, (unsigned)bz);
-    if (es == 2) {
-        if (vec) conv1d_kernel<__nv_bfloat16, true><<<grid, 128, 0, st>>>(p);
-        else conv1d_kernel<__nv_bfloat16, false><<<grid, 128, 0, st>>>(p);
-    } else {
-        if (vec) conv1d_kernel<float, true><<<grid, 128, 0, st>>>(p);
-        else conv1d_kernel<float, false><<<grid, 128, 0, st>>>(p);
-    }
-    return cudaGetLastError();
+    void (*k)(const ConvParams) = es == 2 ? (vec ? conv1d_kernel<__nv_bfloat16, true>
+                                                 : conv1d_kernel<__nv_bfloat16, false>)
+                                          : (vec ? conv1d_kernel<float, true> : conv1d_kernel<float, false>);
+    // a programmatic dependent launch: the grid may start launching while the previous
+    // one in the stream drains; the kernel waits for that grid before it touches memory
+    return launch_dependent(k, grid, dim3(kConvThreads), 0, st, p);
 }
 
 cudaError_t launch_decode(int es, int dstate, const DecodeParams& p, cudaStream_t st) {

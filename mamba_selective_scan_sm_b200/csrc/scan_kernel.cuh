@@ -1,15 +1,16 @@
 // Selective-scan forward kernel for sm_100a.
 //
 // Work split. A CTA owns G channels of one batch row and walks the sequence in
-// tiles of TT steps (TT*sizeof(T) = 64 bytes). Its four warps have two roles:
+// tiles of TT steps (TT*sizeof(T) = 64 or 128 bytes). Its warps have two roles:
 //
-//  * 2 producer warps own the TMA ring and the once-per-(channel, t) prologue. For
+//  * 2 producer warps (6 beside 8 scan warps) own the TMA ring and the
+//    once-per-(channel, t) prologue. For
 //    each tile they wait for the raw tiles (u or the pre-conv x with a 16-byte halo,
 //    dt, z, B, C; B and C are shared by all channels of a batch row), compute
 //    conv + SiLU, delta = softplus(dt + bias), delta*u, D*u and silu(z) into one of
 //    two staging buffers, transpose B and C to fp32 [t][n], and hand the buffer
 //    over through an mbarrier;
-//  * 2 scan warps run the recurrence. The S lanes of a channel each keep NP = NS/S
+//  * SW (2, 3, 4 or 8) scan warps run the recurrence. The S lanes of a channel each keep NP = NS/S
 //    of the (padded) NS states in registers, so a channel's recurrence is spread
 //    over S lanes with no carry between them (A is diagonal: the states never
 //    interact); a lane serves KC channels with the same NP states, so each B and C
@@ -66,7 +67,7 @@ namespace ssm {
 #endif
 
 constexpr int kProWarps = 2;                                // TMA + prologue warps
-constexpr int kProThreads = 32 * kProWarps;                 // 64
+constexpr int kProWarpsWide = 6;                            // with 8 scan warps (one CTA per SM)
 constexpr int kProBarrier = 1;                              // the producers' named barrier
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
@@ -78,7 +79,10 @@ struct ScanCfg {
     static constexpr bool ROWB_NARROW = sizeof(T) == 2 && S == 8 && NP * S == 16 && !VLK &&
                                         SSM_NARROW_ROWB == 128;   // 64-step tiles
     static constexpr int G = SCAN_THREADS / S * KC;   // channels per CTA
-    static constexpr int NT = SCAN_THREADS + kProThreads;   // threads per CTA
+    // producer warps: 2; 6 beside 8 scan warps (d_state 128: one CTA per SM, and the
+    // B/C transposes of 128 states per step are the producers' largest job)
+    static constexpr int PRO_THREADS = 32 * (SW == 8 ? kProWarpsWide : kProWarps);
+    static constexpr int NT = SCAN_THREADS + PRO_THREADS;   // threads per CTA
     // CTAs per SM the launch bounds ask for: three of 6 warps (96 registers per
     // thread), three of 4 warps with two channels per lane (168), five of 4 warps (96);
     // two for d_state 64 / 128 (their B/C tiles take up to 127 KB of shared memory), one
@@ -344,7 +348,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
     if (tid == 0) {
         for (int s = 0; s < NSTAGE; ++s) mbar_init(&full_raw[s], 1);
         for (int s = 0; s < Cfg::NBUF; ++s) {
-            mbar_init(&full_buf[s], kProThreads);
+            mbar_init(&full_buf[s], Cfg::PRO_THREADS);
             mbar_init(&empty_buf[s], kScanThreads);
         }
         fence_mbar_init();
@@ -408,7 +412,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const int l0 = tile_l0(f);
             const bool rv = tile_rev(f);
             const int64_t bL = (int64_t)b * L;
-            for (int e = ptid; e < (SB ? 0 : NS * TT); e += kProThreads) {
+            for (int e = ptid; e < (SB ? 0 : NS * TT); e += Cfg::PRO_THREADS) {
                 const int n = e % NS, row = e / NS, t = l0 + row;
                 const bool ok = n < p.dstate && t >= 0 && t < L;
                 reinterpret_cast<T*>(st + Cfg::RAW_B)[e] =
@@ -419,7 +423,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const int xrows = xpitch / (int)sizeof(T);
             const int xs = (conv && !rv) ? l0 - HALO : l0;
             const int hw = conv ? p.conv_width - 1 : 0;      // history length
-            for (int e = ptid; e < G * xrows; e += kProThreads) {
+            for (int e = ptid; e < G * xrows; e += Cfg::PRO_THREADS) {
                 const int r = e % G, row = e / G, t = xs + row, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 const bool hist = p.conv_hist && !rv && dd < p.dim && t < 0 && t >= -hw;
@@ -428,7 +432,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     ok ? static_cast<const T*>(p.u)[(bL + t) * p.su + dd]
                        : (hist ? static_cast<const T*>(p.conv_hist)[hi] : T(0.f));
             }
-            for (int e = ptid; e < G * TT; e += kProThreads) {
+            for (int e = ptid; e < G * TT; e += Cfg::PRO_THREADS) {
                 const int r = e % G, row = e / G, t = l0 + row, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 reinterpret_cast<T*>(st + Cfg::RAW_DT)[e] =
@@ -445,7 +449,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const bool rv = tile_rev(f);
             const T* gB = static_cast<const T*>(p.Bm) + (int64_t)b * p.dstate * L;
             const T* gC = static_cast<const T*>(p.Cm) + (int64_t)b * p.dstate * L;
-            for (int e = ptid; e < (SB ? 0 : NS * TT); e += kProThreads) {
+            for (int e = ptid; e < (SB ? 0 : NS * TT); e += Cfg::PRO_THREADS) {
                 const int n = e / TT, col = e % TT, t = l0 + col;
                 const bool ok = n < p.dstate && t >= 0 && t < L;
                 const int off = swz<ROWB, SWZ>(n, col * (int)sizeof(T));
@@ -455,7 +459,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             const int xw = xpitch / (int)sizeof(T);
             const int xs = (conv && !rv) ? l0 - HALO : l0;
             const int hw = conv ? p.conv_width - 1 : 0;      // history length
-            for (int e = ptid; e < G * xw; e += kProThreads) {
+            for (int e = ptid; e < G * xw; e += Cfg::PRO_THREADS) {
                 const int r = e / xw, col = e % xw, t = xs + col, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
@@ -466,7 +470,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     ok ? static_cast<const T*>(p.u)[gi]
                        : (hist ? static_cast<const T*>(p.conv_hist)[hi] : T(0.f));
             }
-            for (int e = ptid; e < G * TT; e += kProThreads) {
+            for (int e = ptid; e < G * TT; e += Cfg::PRO_THREADS) {
                 const int r = e / TT, col = e % TT, t = l0 + col, dd = d0 + r;
                 const bool ok = dd < p.dim && t >= 0 && t < L;
                 const int64_t gi = ((int64_t)b * p.dim + dd) * L + t;
@@ -509,9 +513,9 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte chunk
             // steps per producer thread: whole 16-byte chunks, at least one (then not every
             // thread has a segment)
-            constexpr int PER = TT * G / kProThreads;
+            constexpr int PER = TT * G / Cfg::PRO_THREADS;
             constexpr int SEG = PER <= EPC ? EPC : (PER + EPC - 1) / EPC * EPC;
-            static_assert(TT % SEG == 0 && TT * G / SEG <= kProThreads, "segments tile the tile");
+            static_assert(TT % SEG == 0 && TT * G / SEG <= Cfg::PRO_THREADS, "segments tile the tile");
             [[maybe_unused]] constexpr int NSEG = TT * G / SEG;   // segments per tile
             constexpr int SUB = 2 * EPC < SEG ? 2 * EPC : SEG;  // steps per register window
             constexpr int NC = SUB / EPC;                     // dt / z chunks per window
@@ -523,7 +527,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             if constexpr (SB) {
                 // time-invariant B/C: nothing staged per tile
             } else if constexpr (CL) {
-                for (int e = ptid; e < 2 * NCH; e += kProThreads) {
+                for (int e = ptid; e < 2 * NCH; e += Cfg::PRO_THREADS) {
                     const int ten = e / NCH, ch = e % NCH;
                     const uint4 v[1] = {reinterpret_cast<const uint4*>(
                         st + (ten ? Cfg::RAW_C : Cfg::RAW_B))[ch]};
@@ -538,7 +542,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             } else {
                 // (braced: with an unbraced loop as the discarded branch, nvcc 12.9 also
                 // dropped the statement after it, the early return below)
-                for (int e = ptid; e < 2 * NCH; e += kProThreads) {
+                for (int e = ptid; e < 2 * NCH; e += Cfg::PRO_THREADS) {
                     const int ten = e / NCH, ch = e % NCH;
                     const int n = ch % NS, c0 = (ch / NS) * EPC;
                     const uint8_t* src = st + (ten ? Cfg::RAW_C : Cfg::RAW_B) +
@@ -550,7 +554,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     for (int m = 0; m < EPC; ++m) dst[m * NS] = chunk_elem<T>(v, m);
                 }
             }
-            if (NSEG < kProThreads && ptid >= NSEG) return;
+            if (NSEG < Cfg::PRO_THREADS && ptid >= NSEG) return;
             const int r = ptid % G;                           // channel row
             const int t0 = (ptid / G) * SEG;                  // first step of the segment
             const uint4* q4 = reinterpret_cast<const uint4*>(par + (tile_dir(f) * G + r) * 16);
@@ -690,7 +694,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 // The first forward tile's conv halo (positions < 0) landed as zeros;
                 // a continued sequence puts the caller's history there.
                 if (conv && p.conv_hist && p.mode == 0 && chunk == 0 && f == 0)
-                    put_conv_history<T, G, HALO, kProThreads, CL>(p, smem + Cfg::RAW_X, xpitch,
+                    put_conv_history<T, G, HALO, Cfg::PRO_THREADS, CL>(p, smem + Cfg::RAW_X, xpitch,
                                                                    ptid, b, d0);
             } else {
                 // stage 0 was released by every producer at the end of tile f - 1
@@ -700,7 +704,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             // one decision for all producers (this is also the barrier that orders the
             // plain loads and the start mask before the prologue): leave together if a
             // wait ran out
-            if (named_bar_or(kProBarrier, kProThreads, !ok)) {
+            if (named_bar_or(kProBarrier, Cfg::PRO_THREADS, !ok)) {
                 if (USE_TMA && ptid == 0)     // drain the copies still in flight (bounded)
                     for (int g2 = f; g2 < min(f + NSTAGE, nt); ++g2)
                         mbar_wait_bounded(&full_raw[g2 % NSTAGE], (g2 / NSTAGE) & 1);
@@ -714,7 +718,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                 else prologue(FalseT{}, FalseT{}, f, st, buf_of(f));
             }
             mbar_arrive(&full_buf[f & 1]);
-            named_bar_sync(kProBarrier, kProThreads);   // every producer is done with the stage
+            named_bar_sync(kProBarrier, Cfg::PRO_THREADS);   // every producer is done with the stage
             if (USE_TMA && ptid == 0 && f + NSTAGE < nt) issue(f + NSTAGE);
         }
         return;
