@@ -61,6 +61,7 @@ namespace ssm {
 #define SSM_NARROW_ROWB 128
 #endif
 
+
 // Steps whose state-independent operands are prepared together (a divisor of 16).
 #ifndef SSM_SCAN_BATCH
 #define SSM_SCAN_BATCH 2
@@ -122,9 +123,20 @@ struct ScanCfg {
     static constexpr int BUF_P = 0;
     static constexpr int BUF_E = (G / KC) * P_PITCH;
     static constexpr int BUF_BT = BUF_E + G * E_PITCH;
-    static constexpr int BUF_CT = BUF_BT + TT * NS * 4;
+    // B/C staging rows. A producer warp transposing 16-byte chunks writes, per store, the
+    // same n of several rows EPC steps apart; with rows of 16 floats those rows share
+    // banks. So the 2-state splits (8-byte loads) pad each row to NS + 2 floats, and the
+    // splits that load 16 bytes keep NS floats and permute the rows: row t is stored at
+    // t ^ ((t / EPC) & (BCW - 1)), BCW rows per 128 bytes (measured: the long sequence
+    // 1.1 % and the 130M layer 0.9 % faster; the permutation in the 2-state splits slowed
+    // the packed-sequence kernel by 4 %).
+    static constexpr int BCP = NP == 2 ? NS + 2 : NS;   // row pitch (floats)
+    static constexpr int EPC_ = 16 / (int)sizeof(T);
+    static constexpr int BCW = NP % 4 == 0 && BCP < 32 ? (32 / BCP < EPC_ ? 32 / BCP : EPC_) : 1;
+    __host__ __device__ static constexpr int bc_row(int t) { return t ^ ((t / EPC_) & (BCW - 1)); }
+    static constexpr int BUF_CT = BUF_BT + TT * BCP * 4;
     // packed sequences: starts at positions [l0 - HALO, l0 + TT], bit i <-> l0 - HALO + i
-    static constexpr int BUF_META = BUF_CT + TT * NS * 4;
+    static constexpr int BUF_META = BUF_CT + TT * BCP * 4;
     static constexpr int BUF = align_up(BUF_META + 16, 128);
     static constexpr int OFF_BUF = NSTAGE * STAGE;
     static constexpr int OFF_PAR = OFF_BUF + NBUF * BUF;   // [2 directions][G][16] floats
@@ -531,13 +543,22 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     const int ten = e / NCH, ch = e % NCH;
                     const uint4 v[1] = {reinterpret_cast<const uint4*>(
                         st + (ten ? Cfg::RAW_C : Cfg::RAW_B))[ch]};
+                    // chunk ch holds positions ch * EPC .. + EPC - 1 of the [t][n] tile
+                    const int t = ch * EPC / NS, n0 = ch * EPC % NS;
                     float* dst = reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) +
-                                 ch * EPC;
+                                 Cfg::bc_row(t) * Cfg::BCP + n0;
+                    if constexpr (Cfg::BCP == NS) {
 #pragma unroll
-                    for (int m = 0; m < EPC; m += 4)
-                        *reinterpret_cast<float4*>(dst + m) =
-                            make_float4(chunk_elem<T>(v, m), chunk_elem<T>(v, m + 1),
-                                        chunk_elem<T>(v, m + 2), chunk_elem<T>(v, m + 3));
+                        for (int m = 0; m < EPC; m += 4)
+                            *reinterpret_cast<float4*>(dst + m) =
+                                make_float4(chunk_elem<T>(v, m), chunk_elem<T>(v, m + 1),
+                                            chunk_elem<T>(v, m + 2), chunk_elem<T>(v, m + 3));
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < EPC; m += 2)
+                            *reinterpret_cast<float2*>(dst + m) =
+                                make_float2(chunk_elem<T>(v, m), chunk_elem<T>(v, m + 1));
+                    }
                 }
             } else {
                 // (braced: with an unbraced loop as the discarded branch, nvcc 12.9 also
@@ -549,9 +570,10 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                                          swz<ROWB, SWZ>(n, c0 * (int)sizeof(T));
                     const uint4 v[1] = {*reinterpret_cast<const uint4*>(src)};
                     float* dst =
-                        reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) + c0 * NS + n;
+                        reinterpret_cast<float*>(buf + (ten ? Cfg::BUF_CT : Cfg::BUF_BT)) + c0 * Cfg::BCP + n;
+                    const int k = (c0 / EPC) & (Cfg::BCW - 1);   // rows c0 + m land at c0 + (m ^ k)
 #pragma unroll
-                    for (int m = 0; m < EPC; ++m) dst[m * NS] = chunk_elem<T>(v, m);
+                    for (int m = 0; m < EPC; ++m) dst[(m ^ k) * Cfg::BCP] = chunk_elem<T>(v, m);
                 }
             }
             if (NSEG < Cfg::PRO_THREADS && ptid >= NSEG) return;
@@ -955,7 +977,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
             } else if constexpr (NP % 4 == 0) {
 #pragma unroll
                 for (int i = 0; i < NP; i += 4) {
-                    const int o = tt * NS + (i >> 2) * (4 * S);      // slots i .. i + 3
+                    const int o = Cfg::bc_row(tt) * Cfg::BCP + (i >> 2) * (4 * S);   // slots i .. i + 3
                     const float4 b4 = *reinterpret_cast<const float4*>(Bl + o);
                     bv[i] = b4.x; bv[i + 1] = b4.y; bv[i + 2] = b4.z; bv[i + 3] = b4.w;
                     if (!SUMMARY) {
@@ -964,17 +986,17 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     }
                 }
             } else if constexpr (NP == 2) {
-                const float2 b2 = *reinterpret_cast<const float2*>(Bl + tt * NS);
+                const float2 b2 = *reinterpret_cast<const float2*>(Bl + Cfg::bc_row(tt) * Cfg::BCP);
                 bv[0] = b2.x; bv[1] = b2.y;
                 if (!SUMMARY) {
-                    const float2 c2 = *reinterpret_cast<const float2*>(Cl + tt * NS);
+                    const float2 c2 = *reinterpret_cast<const float2*>(Cl + Cfg::bc_row(tt) * Cfg::BCP);
                     cv[0] = c2.x; cv[1] = c2.y;
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    bv[i] = Bl[tt * NS + i];
-                    if (!SUMMARY) cv[i] = Cl[tt * NS + i];
+                    bv[i] = Bl[Cfg::bc_row(tt) * Cfg::BCP + i];
+                    if (!SUMMARY) cv[i] = Cl[Cfg::bc_row(tt) * Cfg::BCP + i];
                 }
             }
         };
