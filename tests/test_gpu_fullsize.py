@@ -92,6 +92,40 @@ def test_fullsize_long_sequence(chunks):
     _check(w, res, inp, _sample(w.batch, w.dim, 8))
 
 
+def test_fullsize_decode_h128_64_steps():
+    """The d_state 128, A-per-head decode workload at full size (the streaming kernel, one
+    wave of CTAs walking 16 KB state tiles), 64 steps, against the oracle on sampled rows."""
+    w = synth.WORKLOADS["decode_h128"]
+    B, D, N, steps, H = w.batch, w.dim, w.dstate, w.steps, w.extra["a_heads"]
+    inp = synth.decode_inputs(B, D, N, steps, 4, "bf16", seed=0, a_heads=H)
+    st = dev(inp["state"])
+    cs = dev(inp["conv_state"], "bf16")
+    X = {k: dev(inp[k], "bf16") for k in ("x", "dt", "z", "B", "C")}
+    P = {k: dev(inp[k]) for k in ("A", "D", "dt_bias", "conv_w", "conv_b")}
+    outs = torch.empty(steps, B, D, dtype=torch.bfloat16, device="cuda")
+    for s in range(steps):
+        ssm.ssm_selective_state_update(st, cs, X["x"][s], X["dt"][s], P["A"], X["B"][s],
+                                       X["C"][s], P["D"], X["z"][s], P["dt_bias"], True,
+                                       P["conv_w"], P["conv_b"], out=outs[s])
+    torch.cuda.synchronize()
+    og, sg = host(outs), host(st)
+    hd = D // H
+    for b, d in _sample(B, D, 16):
+        so = inp["state"][b:b + 1, d:d + 1].astype(np.float64)
+        co = inp["conv_state"][b:b + 1, d:d + 1].astype(np.float64)
+        a_d = inp["A"][d // hd:d // hd + 1]          # the channel's head: one head of one channel
+        yo = []
+        for s in range(steps):
+            sl = lambda k: inp[k][s, b:b + 1, d:d + 1]
+            y, so, co = oracle.state_update(
+                so, co, sl("x"), sl("dt"), a_d, inp["B"][s, b:b + 1], inp["C"][s, b:b + 1],
+                inp["D"][d:d + 1], sl("z"), inp["dt_bias"][d:d + 1], True,
+                inp["conv_w"][d:d + 1], inp["conv_b"][d:d + 1])
+            yo.append(y[0, 0])
+        assert_close_out(og[:, b, d], np.array(yo), "bf16", f"decode channel {(b, d)}")
+        state_close(sg[b, d], so[0, 0], "state")
+
+
 def test_fullsize_decode_64_steps():
     w = synth.WORKLOADS["decode"]
     B, D, N, steps = w.batch, w.dim, w.dstate, w.steps
