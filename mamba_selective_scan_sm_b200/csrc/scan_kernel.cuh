@@ -131,6 +131,10 @@ struct ScanCfg {
     // 1.1 % and the 130M layer 0.9 % faster; the permutation in the 2-state splits slowed
     // the packed-sequence kernel by 4 %).
     static constexpr int BCP = NP == 2 ? NS + 2 : NS;   // row pitch (floats)
+    // The prologue's SiLUs take the reciprocal on the FMA pipe (one SFU op per value) in
+    // the 8 x 2 split, where the SFU is the busiest pipe (the 130M layer: 230 -> 226 µs);
+    // elsewhere the SFU reciprocal measured faster.
+    static constexpr bool SILU_FMA = NP == 8 && S == 2;
     static constexpr int EPC_ = 16 / (int)sizeof(T);
     static constexpr int BCW = NP % 4 == 0 && BCP < 32 ? (32 / BCP < EPC_ ? 32 / BCP : EPC_) : 1;
     __host__ __device__ static constexpr int bc_row(int t) { return t ^ ((t / EPC_) & (BCW - 1)); }
@@ -661,7 +665,7 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                             }
                             acc = fma2(w2[k], pk2(xa, xb), acc);
                         }
-                        u2 = silu2(acc);
+                        u2 = Cfg::SILU_FMA ? silu2_fma<sizeof(T) == 2 ? 2 : 3>(acc) : silu2(acc);
                     } else {
                         u2 = pk2(X(i), X(i + 1));
                     }
@@ -678,7 +682,10 @@ scan_fwd_kernel(const __grid_constant__ ScanMaps maps, const ScanParams p) {
                     }
                     if (!SUMMARY) {
                         uint64_t g2 = pk2(1.f, 1.f);
-                        if (has_z) g2 = silu2(pk2(ZV(i), ZV(i + 1)));
+                        if (has_z) {
+                            const uint64_t z2 = pk2(ZV(i), ZV(i + 1));
+                            g2 = Cfg::SILU_FMA ? silu2_fma<sizeof(T) == 2 ? 2 : 3>(z2) : silu2(z2);
+                        }
                         const float2 g = upk2(g2), dv = upk2(mul2(D2, u2));
                         *reinterpret_cast<float4*>(erow + i * 8) = make_float4(dv.x, g.x, dv.y, g.y);
                     }
